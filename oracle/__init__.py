@@ -1,0 +1,147 @@
+"""CPU oracle for the I2_S ternary linear layer -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps the plain C oracle
+(``bitnet_oracle.c``; readings R1-R4 are stated in ``bitnet_oracle.h``) with
+numpy-friendly functions.  It shares no code with the CUDA library.
+"""
+import ctypes as _C
+
+import numpy as _np
+
+from .build import build as _build
+
+OK, NONFINITE, NOT_TERNARY, OVERFLOW = 0, 1, 2, 4
+
+_lib = _C.CDLL(_build())
+_i64, _f32 = _C.c_int64, _C.c_float
+_P = _C.c_void_p
+for _name, _args, _ret in [
+    ("oracle_blocks", [_i64], _i64),
+    ("oracle_kpad", [_i64], _i64),
+    ("oracle_quant_act", [_P, _i64, _i64, _P, _P], _C.c_int),
+    ("oracle_pack", [_P, _i64, _i64, _P], _C.c_int),
+    ("oracle_unpack", [_P, _i64, _i64, _P], None),
+    ("oracle_unpack_misread64", [_P, _i64, _i64, _P], None),
+    ("oracle_ternary_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
+    ("oracle_dequant", [_P, _P, _f32, _i64, _i64, _P, _P], None),
+    ("oracle_linear", [_P, _i64, _i64, _P, _i64, _f32, _P, _P, _P], _C.c_int),
+    ("oracle_linear_rows", [_P, _i64, _i64, _P, _i64, _f32, _P, _i64, _P, _P], _C.c_int),
+]:
+    _fn = getattr(_lib, _name)
+    _fn.argtypes, _fn.restype = _args, _ret
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_P)
+
+
+def _c(a, dtype):
+    return _np.ascontiguousarray(a, dtype=dtype)
+
+
+def blocks(k: int) -> int:
+    return int(_lib.oracle_blocks(k))
+
+
+def kpad(k: int) -> int:
+    return int(_lib.oracle_kpad(k))
+
+
+def packed_row_bytes(k: int) -> int:
+    return 32 * blocks(k)
+
+
+def quant_act(x):
+    """x fp32 [m,k] -> (q int8 [m,kpad], s_act fp32 [m], status)."""
+    x = _c(x, _np.float32)
+    m, k = x.shape
+    q = _np.empty((m, kpad(k)), _np.int8)
+    s = _np.empty((m,), _np.float32)
+    st = _lib.oracle_quant_act(_ptr(x), m, k, _ptr(q), _ptr(s))
+    return q, s, st
+
+
+def pack(w):
+    """w int8 [n,k] in {-1,0,1} -> (packed uint8 [n, 32*blocks], status)."""
+    w = _c(w, _np.int8)
+    n, k = w.shape
+    p = _np.empty((n, packed_row_bytes(k)), _np.uint8)
+    st = _lib.oracle_pack(_ptr(w), n, k, _ptr(p))
+    return p, st
+
+
+def unpack(packed, k):
+    packed = _c(packed, _np.uint8)
+    n = packed.shape[0]
+    w = _np.empty((n, k), _np.int8)
+    _lib.oracle_unpack(_ptr(packed), n, k, _ptr(w))
+    return w
+
+
+def unpack_misread64(packed, k):
+    """The planted 64-element misreading (mutation test only)."""
+    packed = _c(packed, _np.uint8)
+    n = packed.shape[0]
+    w = _np.empty((n, k), _np.int8)
+    _lib.oracle_unpack_misread64(_ptr(packed), n, k, _ptr(w))
+    return w
+
+
+def ternary_matmul(q, packed, k):
+    """q int8 [m,kpad] x packed [n,...] -> (acc int32 [m,n], status)."""
+    q = _c(q, _np.int8)
+    packed = _c(packed, _np.uint8)
+    m, n = q.shape[0], packed.shape[0]
+    acc = _np.empty((m, n), _np.int32)
+    st = _lib.oracle_ternary_matmul(_ptr(q), m, _ptr(packed), n, k, _ptr(acc))
+    return acc, st
+
+
+def dequant(acc, s_act, s_w):
+    """-> (y64 fp64 [m,n], y32 fp32 [m,n])."""
+    acc = _c(acc, _np.int32)
+    s_act = _c(s_act, _np.float32)
+    m, n = acc.shape
+    y64 = _np.empty((m, n), _np.float64)
+    y32 = _np.empty((m, n), _np.float32)
+    _lib.oracle_dequant(_ptr(acc), _ptr(s_act), float(s_w), m, n, _ptr(y64), _ptr(y32))
+    return y64, y32
+
+
+def linear(x, packed, n, k, s_w):
+    """Whole layer -> (acc int32, y64 fp64, y32 fp32, status)."""
+    x = _c(x, _np.float32)
+    packed = _c(packed, _np.uint8)
+    m = x.shape[0]
+    acc = _np.empty((m, n), _np.int32)
+    y64 = _np.empty((m, n), _np.float64)
+    y32 = _np.empty((m, n), _np.float32)
+    st = _lib.oracle_linear(_ptr(x), m, k, _ptr(packed), n, float(s_w),
+                            _ptr(acc), _ptr(y64), _ptr(y32))
+    return acc, y64, y32, st
+
+
+def linear_rows(x, packed, n, k, s_w, rows):
+    """Only the output columns ``rows`` -> (acc int32 [m,cnt], y64 [m,cnt], status)."""
+    x = _c(x, _np.float32)
+    packed = _c(packed, _np.uint8)
+    idx = _c(rows, _np.int64)
+    m, cnt = x.shape[0], idx.shape[0]
+    acc = _np.empty((m, cnt), _np.int32)
+    y64 = _np.empty((m, cnt), _np.float64)
+    st = _lib.oracle_linear_rows(_ptr(x), m, k, _ptr(packed), n, float(s_w),
+                                 _ptr(idx), cnt, _ptr(acc), _ptr(y64))
+    return acc, y64, st
+
+
+def linear_stack(xs, packed_list, shapes, scales):
+    """Loops the layers in order: xs[i] is the fp32 input of layer i (aliasing
+    allowed), shapes[i] = (n, k).  Returns lists (acc, y64, status)."""
+    accs, ys, st = [], [], 0
+    for x, p, (n, k), s in zip(xs, packed_list, shapes, scales):
+        a, y64, _, s1 = linear(x, p, n, k, s)
+        accs.append(a)
+        ys.append(y64)
+        st |= s1
+    return accs, ys, st

@@ -1,0 +1,295 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself:
+hand-derived worked examples (tests/golden), closed forms, invariants, brute
+force over the unpacked ternary matrix, and a planted-mistake check.
+
+Readings pinned here (stated in oracle/bitnet_oracle.h):
+R1 activation quantiser, R2 packed layout, R3 codes and tail, R4 linear.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from ternary_weight_i2_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------- quantiser R1
+
+def _read_quant_golden():
+    cases, cur = [], {}
+    with open(os.path.join(GOLDEN, "quant_small.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = line.split(":", 1)
+            cur[key] = val.split()
+            if key == "s":
+                cases.append(cur)
+                cur = {}
+    return cases
+
+
+def test_quant_golden_examples():
+    cases = _read_quant_golden()
+    assert len(cases) == 4
+    for c in cases:
+        x = np.array([float(v) for v in c["x"]], np.float32)[None, :]
+        want = np.array([int(v) for v in c["q"]], np.int8)
+        num, den = c["s"][0].split("/")
+        s_want = np.float32(np.float32(float(num)) / np.float32(float(den)))
+        q, s, st = oracle.quant_act(x)
+        assert st == oracle.OK
+        np.testing.assert_array_equal(q[0, : x.shape[1]], want)
+        assert s[0] == s_want
+
+
+def test_quant_invariants_random():
+    rng = np.random.default_rng(1)
+    for k in (1, 7, 128, 300, 1536):
+        x = synth.normal_outliers(rng, 9, k)
+        x[3] *= np.float32(1e-6)
+        x[4] *= np.float32(1e6)
+        q, s, st = oracle.quant_act(x)
+        assert st == oracle.OK
+        kp = oracle.kpad(k)
+        assert q.shape == (9, kp)
+        assert not q[:, k:].any()                         # zero padding
+        qv = q[:, :k].astype(np.int64)
+        assert np.abs(qv).max() <= 127 and qv.min() >= -127  # never -128
+        amax = np.abs(x).max(axis=1)
+        for r in range(9):
+            i = int(np.argmax(np.abs(x[r])))
+            assert abs(int(qv[r, i])) == 127                 # absmax maps to 127
+            sgn = np.sign(qv[r])
+            assert np.all((sgn == 0) | (sgn == np.sign(x[r])))
+            assert s[r] == np.float32(amax[r] / np.float32(127))
+            err = np.abs(qv[r] * np.float64(s[r]) - x[r].astype(np.float64))
+            assert err.max() <= 0.5 * float(s[r]) * (1 + 1e-4)
+
+
+def test_quant_special_rows():
+    x = np.zeros((6, 200), np.float32)
+    x[0] = 3.0                     # constant positive
+    x[1] = -2.0                    # constant negative
+    # row 2 stays zero
+    x[3] = 1.0
+    x[3, 17] = np.nan              # non-finite row
+    x[4] = 1.0
+    x[4, 5] = np.inf               # non-finite row
+    x[5, :4] = [1e-38, -5e-39, 0.0, 2e-39]   # 127/amax overflows to inf
+    q, s, st = oracle.quant_act(x)
+    assert st == oracle.NONFINITE
+    assert (q[0, :200] == 127).all() and (q[1, :200] == -127).all()
+    assert not q[2].any() and s[2] == 0
+    assert not q[3].any() and s[3] == 0
+    assert not q[4].any() and s[4] == 0
+    assert list(q[5, :5]) == [127, -127, 0, 127, 0]
+
+
+def test_quant_ties_round_half_even_constructed():
+    # amax = 127 makes inv exactly 1, so x*inv = x: every half rounds to even
+    halves = np.arange(-126.5, 127.0, 1.0, dtype=np.float32)
+    x = np.concatenate([halves, [np.float32(127.0)]])[None, :]
+    q, _, _ = oracle.quant_act(x)
+    # half-even: floor if floor is even, else ceil
+    fl = np.floor(halves).astype(np.int64)
+    exp = np.where(fl % 2 == 0, fl, fl + 1)
+    np.testing.assert_array_equal(q[0, : halves.size].astype(np.int64), exp)
+
+
+# ------------------------------------------------------- pack layout R2, R3
+
+def _read_pack_golden():
+    spec = {}
+    with open(os.path.join(GOLDEN, "pack_k130.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                spec[key] = val.split()
+    return spec
+
+
+def test_pack_golden_bytes():
+    spec = _read_pack_golden()
+    k = int(spec["K"][0])
+    w = np.zeros((1, k), np.int8)
+    for item in spec["w"]:
+        pos, val = item.split(":")
+        w[0, int(pos)] = int(val)
+    want = None
+    for item in spec["bytes"]:
+        pos, val = item.split(":")
+        if pos == "default":
+            want = np.full(32 * ((k + 127) // 128), int(val, 16), np.uint8)
+    for item in spec["bytes"]:
+        pos, val = item.split(":")
+        if pos != "default":
+            want[int(pos)] = int(val, 16)
+    p, st = oracle.pack(w)
+    assert st == oracle.OK
+    np.testing.assert_array_equal(p[0], want)
+
+
+@pytest.mark.parametrize("k", list(range(1, 301, 1)) + [1535, 8960, 9024])
+def test_pack_unpack_roundtrip_and_tail(k):
+    rng = np.random.default_rng(k)
+    w = synth.ternary(rng, 3, k, (0.3, 0.4, 0.3))
+    p, st = oracle.pack(w)
+    assert st == oracle.OK
+    assert p.shape == (3, 32 * ((k + 127) // 128))
+    np.testing.assert_array_equal(oracle.unpack(p, k), w)
+    # every 2-bit field of a position k' >= K holds code 01 (weight 0)
+    kp = oracle.kpad(k)
+    for kk in range(k, kp):
+        byte = 32 * (kk // 128) + kk % 32
+        sh = 2 * ((kk % 128) // 32)
+        assert ((p[:, byte] >> sh) & 3 == 1).all()
+    # no field anywhere holds the unused code 3
+    for sh in (0, 2, 4, 6):
+        assert not (((p >> sh) & 3) == 3).any()
+
+
+def test_pack_rejects_non_ternary():
+    w = np.zeros((2, 10), np.int8)
+    w[1, 3] = 2
+    w[0, 9] = -128
+    p, st = oracle.pack(w)
+    assert st == oracle.NOT_TERNARY
+    np.testing.assert_array_equal(oracle.unpack(p, 10), np.zeros((2, 10), np.int8))
+
+
+def _onehot_check(unpacker, k, k0s):
+    """For each k0, a row holding a single +1 at k0 must decode to that row."""
+    bad = 0
+    for k0 in k0s:
+        w = np.zeros((1, k), np.int8)
+        w[0, k0] = 1
+        p, _ = oracle.pack(w)
+        bad += int(not np.array_equal(unpacker(p, k), w))
+    return bad
+
+
+def test_onehot_gather_layout():
+    k = 300
+    rng = np.random.default_rng(5)
+    x = synth.normal(rng, 3, k)
+    q, s, _ = oracle.quant_act(x)
+    for k0 in range(k):
+        w = np.zeros((1, k), np.int8)
+        w[0, k0] = 1
+        p, _ = oracle.pack(w)
+        acc, st = oracle.ternary_matmul(q, p, k)
+        assert st == oracle.OK
+        np.testing.assert_array_equal(acc[:, 0], q[:, k0].astype(np.int32))
+
+
+def test_misread64_is_caught():
+    """The planted 64-element misreading keeps every 128-span's multiset of
+    weights (so sums and non-zero counts agree) but fails the one-hot check."""
+    k = kf = 8960
+    rng = np.random.default_rng(11)
+    w = synth.ternary(rng, 4, k)
+    p, _ = oracle.pack(w)
+    wm = oracle.unpack_misread64(p, k)
+    for j in range(kf // 128):
+        a = np.sort(w[:, 128 * j:128 * (j + 1)], axis=1)
+        b = np.sort(wm[:, 128 * j:128 * (j + 1)], axis=1)
+        np.testing.assert_array_equal(a, b)
+    assert not np.array_equal(wm, w[:, :kf])
+    assert _onehot_check(oracle.unpack_misread64, 256, range(256)) > 0
+    assert _onehot_check(oracle.unpack, 256, range(256)) == 0
+
+
+# ------------------------------------------------------------- linear R4
+
+@pytest.mark.parametrize("m,n,k", [(1, 1, 1), (2, 3, 5), (5, 9, 127), (3, 9, 128),
+                                   (4, 7, 129), (5, 2, 300), (1, 9, 256), (2, 4, 1536)])
+def test_linear_matches_bruteforce(m, n, k):
+    rng = np.random.default_rng(100 * m + n + k)
+    w = synth.ternary(rng, n, k)
+    x = synth.normal_outliers(rng, m, k)
+    s_w = synth.weight_scale(rng)
+    p, _ = oracle.pack(w)
+    acc, y64, y32, st = oracle.linear(x, p, n, k, s_w)
+    assert st == oracle.OK
+    q, s_act, _ = oracle.quant_act(x)
+    ref = q[:, :k].astype(np.float64) @ w.astype(np.float64).T   # exact integers
+    np.testing.assert_array_equal(acc.astype(np.float64), ref)
+    # y against the double-precision sum of dequantised products
+    yd = (q[:, :k].astype(np.float64) * np.float64(1) * s_act[:, None].astype(np.float64)) @ \
+         (w.astype(np.float64) * np.float64(s_w)).T
+    np.testing.assert_allclose(y64, yd, rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(y32, y64, rtol=1e-6, atol=0)
+
+
+def test_linear_special_rows_closed_forms():
+    k, n, m = 1000, 4, 3
+    rng = np.random.default_rng(2)
+    x = synth.normal(rng, m, k)
+    w = np.zeros((n, k), np.int8)
+    w[1] = 1
+    w[2] = -1
+    w[3] = synth.ternary(rng, 1, k)[0]
+    p, _ = oracle.pack(w)
+    acc, y64, _, _ = oracle.linear(x, p, n, k, 0.05)
+    q, _, _ = oracle.quant_act(x)
+    sq = q[:, :k].astype(np.int64).sum(axis=1)
+    assert (acc[:, 0] == 0).all() and (y64[:, 0] == 0).all()
+    np.testing.assert_array_equal(acc[:, 1], sq)
+    np.testing.assert_array_equal(acc[:, 2], -sq)
+    # zero weights contribute nothing: zeroing weight (3, i) moves acc by -w*q
+    for i in rng.choice(k, 20, replace=False):
+        w2 = w.copy()
+        w2[3, i] = 0
+        p2, _ = oracle.pack(w2)
+        acc2, _, _, _ = oracle.linear(x, p2, n, k, 0.05)
+        np.testing.assert_array_equal(acc2[:, 3] - acc[:, 3],
+                                      -int(w[3, i]) * q[:, i].astype(np.int32))
+        np.testing.assert_array_equal(acc2[:, :3], acc[:, :3])
+
+
+def test_linear_saturation_max_k():
+    k = 9024
+    x = np.full((2, k), 3.25, np.float32)
+    x[1] = -3.25
+    w = np.ones((2, k), np.int8)
+    w[1] = -1
+    p, _ = oracle.pack(w)
+    acc, _, _, st = oracle.linear(x, p, 2, k, 0.1)
+    assert st == oracle.OK
+    assert acc[0, 0] == 127 * 9024 == 1146048
+    assert acc[0, 1] == -1146048 and acc[1, 0] == -1146048 and acc[1, 1] == 1146048
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 7, 8, 13, 64])
+def test_linear_rows_independent_of_m(m):
+    """Remainder rows (M = 4, 5, ... as in the blog post's third bug) give the
+    same result as computing each token alone."""
+    k, n = 257, 33
+    rng = np.random.default_rng(m)
+    w = synth.ternary(rng, n, k)
+    x = synth.normal_outliers(rng, m, k)
+    p, _ = oracle.pack(w)
+    acc, y64, _, _ = oracle.linear(x, p, n, k, 0.02)
+    for r in range(m):
+        a1, y1, _, _ = oracle.linear(x[r:r + 1], p, n, k, 0.02)
+        np.testing.assert_array_equal(acc[r], a1[0])
+        np.testing.assert_array_equal(y64[r], y1[0])
+
+
+def test_linear_rows_sampled_equals_full():
+    k, n, m = 8960, 40, 2
+    rng = np.random.default_rng(9)
+    w = synth.ternary(rng, n, k)
+    x = synth.normal_outliers(rng, m, k)
+    p, _ = oracle.pack(w)
+    acc, y64, _, _ = oracle.linear(x, p, n, k, 0.07)
+    idx = np.array([0, 5, 39, 17])
+    a2, y2, _ = oracle.linear_rows(x, p, n, k, 0.07, idx)
+    np.testing.assert_array_equal(a2, acc[:, idx])
+    np.testing.assert_array_equal(y2, y64[:, idx])
