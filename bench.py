@@ -1,0 +1,424 @@
+"""Benchmark of the ternary linear-stack decode path on B200.
+
+Workload: the 28-layer stack of a 1.5B-class decoder's seven ternary linears
+(q, k, v, o 1536x1536/256; gate, up 1536->8960; down 8960->1536), 1.31e9
+ternary weights = 327,548,928 packed bytes, M = 1 token per step by default,
+per-token int8 activation quantisation fused before every GEMV.  One step is
+one bitnet_linear_stack launch over all 196 layers.  Weights (327.5 MB) are
+larger than the 126 MB L2, so every step streams them from HBM; no L2 flush is
+needed between steps.
+
+Prints one JSON line (rank 0).  `value` is whole-job tokens/s with inputs
+resident in HBM; `e2e` is the same metric through the C ABI with the step's
+activations copied host->device and the outputs device->host every step.
+Multi-GPU runs are independent replicas (the path has no exchange step).
+
+``--impl reference`` times the CPU oracle (plain single-threaded C) on the
+same workload instead: each step is one M=1 token through a bounded sample of
+the stack's layers.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "M=1 ternary linear-stack tokens/s & packed-weight HBM GB/s; prefill int8 TOPS"
+STACK_BYTES = 327_548_928
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--m", type=int, default=1, help="tokens per step (1, 2, 4, 8)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the M = 2, 4, 8 lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured", d
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback", {}
+
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemv.cu", "gemv.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "ternary_weight_i2_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(m):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "gemv_stack_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("source_hash") == _kernel_source_hash() and str(m) in d.get("bytes_per_launch", {}):
+            return float(d["bytes_per_launch"][str(m)])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def build_stack(m, dev):
+    """Pack the 28 layers on the GPU; return descriptors, the contiguous input
+    and output buffers and their per-layer views."""
+    import torch
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import synth
+
+    packed, tws = [], []
+    for L in range(synth.NUM_LAYERS):
+        for (name, n, k), (w, s) in zip(synth.LAYER_SHAPES, synth.layer_weights(L, 3)):
+            wt = torch.from_numpy(w).to(dev)
+            pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
+            fl = torch.zeros(1, dtype=torch.int32, device=dev)
+            tw2.pack_ternary(wt, pk, flags=fl)
+            del wt
+            packed.append(pk)
+            tws.append(tw2.make_tw(pk, n, k, s))
+    torch.cuda.synchronize()
+    # all distinct inputs in one buffer, all outputs in another
+    in_sizes = [m * k for _ in range(synth.NUM_LAYERS) for k in synth.LAYER_INPUT_K]
+    out_sizes = [m * n for _ in range(synth.NUM_LAYERS) for (_, n, _) in synth.LAYER_SHAPES]
+    x_host = np.empty(sum(in_sizes), np.float32)
+    off = 0
+    for L in range(synth.NUM_LAYERS):
+        for a in synth.layer_inputs(L, m, 3):
+            x_host[off:off + a.size] = a.ravel()
+            off += a.size
+    x_dev = torch.from_numpy(x_host).to(dev)
+    y_dev = torch.empty(sum(out_sizes), dtype=torch.float32, device=dev)
+    xs, ys, off, yoff = [], [], 0, 0
+    for L in range(synth.NUM_LAYERS):
+        views = []
+        for k in synth.LAYER_INPUT_K:
+            views.append(x_dev[off:off + m * k].view(m, k))
+            off += m * k
+        for (_, n, _), j in zip(synth.LAYER_SHAPES, synth.LAYER_INPUT_OF):
+            xs.append(views[j])
+            ys.append(y_dev[yoff:yoff + m * n].view(m, n))
+            yoff += m * n
+    return packed, tws, xs, ys, x_host, x_dev, y_dev
+
+
+def time_device(call, steps, warmup, stream):
+    """Per-launch CUDA-event durations on `stream` and the whole-loop time."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    _barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        starts[i].record(stream)
+        call()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    _barrier()
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total = starts[0].elapsed_time(ends[-1])
+    return total, per
+
+
+def _barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def _max_over_ranks(v):
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return v
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import build as tbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    tbuild.build()
+    tw2.load()
+
+    m = args.m
+    packed, tws, xs, ys, x_host, x_dev, y_dev = build_stack(m, dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    call = tw2.StackCall(xs, tws, ys)
+    stream = torch.cuda.current_stream()
+
+    # device-resident timing through a captured graph of the stack launch
+    call(flags=flags)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(flags=flags)
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms, per = time_device(graph.replay, args.steps, args.warmup, stream)
+    clk = clocks.stop()
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"device flags {int(flags.item())} during the timed run")
+    total_ms = _max_over_ranks(total_ms)
+    kern_ms = _max_over_ranks(statistics.mean(per))
+    ms_step = total_ms / args.steps
+    tok_s = world * m / (ms_step * 1e-3)
+
+    # end to end through the C ABI: H2D inputs, stack call, D2H outputs per step
+    e2e = None
+    if not args.no_e2e:
+        x_pin = torch.from_numpy(x_host).pin_memory()
+        y_pin = torch.empty(y_dev.numel(), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            x_dev.copy_(x_pin, non_blocking=True)
+            call(flags=flags)
+            y_pin.copy_(y_dev, non_blocking=True)
+
+        e_total, _ = time_device(e2e_step, max(args.steps // 2, 10), args.warmup, stream)
+        e_total = _max_over_ranks(e_total)
+        e_steps = max(args.steps // 2, 10)
+        e2e = {"value": world * m / (e_total / e_steps * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(x_host.nbytes), "d2h_bytes_per_step": int(y_dev.numel() * 4)}
+
+    peak, peak_kind, peaks = _peaks()
+    achieved = STACK_BYTES / (kern_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": _ncu_traffic(m),
+                "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "kernel": "gemv_stack_kernel", "kernel_ms": round(kern_ms, 5),
+                "algorithmic_bytes": STACK_BYTES}
+
+    sweep = {}
+    if not args.no_sweep and m == 1:
+        for ms in (2, 4, 8):
+            _, twsm, xsm, ysm, _, _, _ = build_stack_views(ms, dev, tws)
+            c2 = tw2.StackCall(xsm, twsm, ysm)
+            c2(flags=flags)
+            t2, per2 = time_device(lambda: c2(flags=flags), 50, 5, stream)
+            t2 = _max_over_ranks(t2)
+            k2 = _max_over_ranks(statistics.mean(per2))
+            sweep[str(ms)] = {"tokens_per_s": round(world * ms / (t2 / 50 * 1e-3), 1),
+                              "weight_gbs": round(STACK_BYTES / (k2 * 1e-3) / 1e9, 1)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(budget_s=12.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(tok_s, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+            "data": "synthetic (seeded ternary weights and fp32 activations, BASELINE shapes)",
+            "config": {"workload": "28-layer ternary linear stack, 196 layers, M=%d decode" % m,
+                       "tokens_per_step_per_gpu": m, "layers": 196,
+                       "packed_weight_bytes": STACK_BYTES,
+                       "l2": "weights 327.5 MB > 126 MB L2 (no flush needed)",
+                       "parallelism": "replicas" if world > 1 else "single GPU",
+                       "timing": "CUDA graph replay of one bitnet_linear_stack launch per step"},
+            "weight_gbs": round(STACK_BYTES * world / (ms_step * 1e-3) / 1e9, 1),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "m_sweep": sweep,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def build_stack_views(m, dev, tws):
+    """Inputs/outputs for another token count, reusing the packed weights."""
+    import torch
+    from ternary_weight_i2_b200 import synth
+    xs, ys = [], []
+    for L in range(synth.NUM_LAYERS):
+        views = [torch.from_numpy(a).to(dev) for a in synth.layer_inputs(L, m, 3)]
+        for (_, n, _), j in zip(synth.LAYER_SHAPES, synth.LAYER_INPUT_OF):
+            xs.append(views[j])
+            ys.append(torch.empty((m, n), dtype=torch.float32, device=dev))
+    return None, tws, xs, ys, None, None, None
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+class OracleSample:
+    """A bounded sample of the workload for the CPU oracle: decoder layer 0's
+    seven linears (11.7 MB packed, 1/28 of the stack) at M = 1, packed once by
+    the oracle.  One pass = one token through those seven layers."""
+
+    def __init__(self):
+        import oracle
+        from ternary_weight_i2_b200 import synth
+        self.oracle = oracle
+        xl = synth.layer_inputs(0, 1, 3)
+        self.layers = []
+        self.bytes = 0
+        for (name, n, k), (w, s), j in zip(synth.LAYER_SHAPES, synth.layer_weights(0, 3),
+                                           synth.LAYER_INPUT_OF):
+            pk, _ = oracle.pack(w)
+            self.layers.append((xl[j], pk, n, k, s))
+            self.bytes += pk.nbytes
+
+    def run(self):
+        t0 = time.perf_counter()
+        for x, pk, n, k, s in self.layers:
+            self.oracle.linear(x, pk, n, k, s)
+        return time.perf_counter() - t0
+
+    def tokens_per_s(self, secs, passes):
+        # fraction of the stack per pass = self.bytes / STACK_BYTES
+        return passes * (self.bytes / STACK_BYTES) / secs
+
+
+def cpu_baseline(budget_s=12.0):
+    smp = OracleSample()
+    secs, passes = 0.0, 0
+    while secs < budget_s:
+        secs += smp.run()
+        passes += 1
+    return {"value": round(smp.tokens_per_s(secs, passes), 4), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{passes} passes of one M=1 token through decoder layer 0's seven linears "
+                      f"({smp.bytes} of {STACK_BYTES} packed bytes per pass, {secs:.1f} s single-threaded), "
+                      f"scaled by packed bytes to the 196-layer stack"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    smp = OracleSample()
+    for _ in range(args.warmup):
+        smp.run()
+    t_total = 0.0
+    for _ in range(args.steps):
+        t_total += smp.run()
+    tok_s = smp.tokens_per_s(t_total, args.steps)
+    ms_step = t_total / args.steps * 1e3 * STACK_BYTES / smp.bytes
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(tok_s, 4), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": {"workload": "28-layer ternary linear stack, 196 layers, M=1 decode",
+                   "tokens_per_step_per_gpu": 1},
+        "cpu_baseline": {"value": round(tok_s, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: one M=1 token through decoder layer 0's seven linears "
+                                   f"({smp.bytes} packed bytes, 1/28 of the stack) on the plain C oracle, "
+                                   f"single-threaded; tokens/s scaled by packed bytes to the full stack"},
+        "e2e": {"value": round(tok_s, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+/*
+ * bitnet.h -- C ABI of the B200 (sm_100a) I2_S ternary linear-layer library.
+ *
+ * The operation ("VibeVoice-ASR-BitNet Technical Report", §2.2.2 and §2.4.2,
+ * Figure 4): a linear layer y = x W^T whose weights W [N,K] take values in
+ * {-1, 0, +1} and are stored 2 bits each, grouped 128 elements per block (the
+ * grouping the ARM debugging blog post "Paper 說支援 ARM，我大概是第一個真的去編譯
+ * 的人" establishes in its second postscript), with one fp32 scale s_w per
+ * tensor; activations x [M,K] are quantised per token to int8 by absmax/127 at
+ * run time, multiplied against the ternary weights with exact int32
+ * accumulation, and the sums are dequantised in fp32.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named d_* or documented "device" point to CUDA device memory of
+ *   the current device; the caller owns every buffer.  Functions that take a
+ *   workspace never allocate; no function allocates device memory per call.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  All GPU work is
+ *   enqueued on it and the functions return without synchronising.
+ * - Errors found on the host (bad argument, misaligned pointer, device that is
+ *   not sm_100) are returned synchronously and nothing is enqueued.  A
+ *   function never returns BITNET_OK without doing its work.
+ * - Conditions found on the GPU are OR-ed as BITNET_FLAG_* bits into the
+ *   int32 word *d_flags (device memory, nullable); read it after the stream
+ *   has been synchronised.  bitnet_status_from_flags() maps it to a status.
+ * - Layouts are row-major and dense: x [M,K] fp32, y [M,N] fp32, int32
+ *   acc [M,N], int8 w [N,K], packed [N, 32*ceil(K/128)] bytes.
+ *
+ * Packed format (readings of points the pages leave open)
+ * ---------------------------------------------------------
+ * Row n of the packed matrix holds 32*ceil(K/128) bytes.  Element
+ * k = 128*j + 32*g + b (g = 0..3, b = 0..31) is the 2-bit field at bits
+ * [2g, 2g+1] of byte 32*j + b; the field holds w + 1 (00 = -1, 01 = 0,
+ * 10 = +1); fields of positions k >= K hold 01.  The weight scale is not in the
+ * buffer: it travels in bitnet_tw.  Compatibility with other I2_S files is not
+ * claimed.
+ *
+ * Activation quantiser (per token m, fp32, no fused multiply-add)
+ * ---------------------------------------------------------------
+ * amax = max_k |x[m,k]|; a row holding NaN or Inf gives codes 0 and scale 0 and
+ * raises BITNET_FLAG_NONFINITE; amax == 0 gives codes 0 and scale 0; otherwise
+ * inv = 127/amax, q = 0 where x == 0, else clamp(rint(x*inv), -127, 127)
+ * (round half to even), and scale = amax/127.  Pads k >= K of int8 rows are 0.
+ *
+ * Linear
+ * ------
+ * acc[m,n] = sum_k q[m,k] * w[n,k] (exact int32);
+ * y[m,n] = ((float)acc[m,n] * s_act[m]) * s_w, two rounded fp32 products.
+ */
+#ifndef BITNET_H
+#define BITNET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BITNET_API __attribute__((visibility("default")))
+#else
+#define BITNET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,        /* null/negative/misaligned/oversized argument   */
+    BITNET_ERR_NOT_TERNARY = 2,        /* a weight outside {-1,0,+1} (device flag)      */
+    BITNET_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 (B200)           */
+    BITNET_ERR_CUDA = 4,               /* a CUDA runtime call failed                    */
+    BITNET_ERR_NONFINITE = 5,          /* an activation row held NaN/Inf (device flag)  */
+    BITNET_ERR_TIMEOUT = 6,            /* a bounded device-side wait ran out (flag)     */
+    BITNET_ERR_WORKSPACE = 7           /* the workspace given is too small              */
+} bitnet_status;
+
+/* Bits OR-ed into *d_flags by the kernels. */
+#define BITNET_FLAG_NOT_TERNARY 0x1
+#define BITNET_FLAG_NONFINITE   0x2
+#define BITNET_FLAG_TIMEOUT     0x4
+
+/* One ternary weight tensor as produced by bitnet_pack_ternary.
+ * packed: device pointer, 16-byte aligned, [n, 32*ceil(k/128)] bytes;
+ * n, k: output and input widths (1 <= k <= BITNET_MAX_K, n >= 1);
+ * scale: the per-tensor fp32 weight scale s_w. */
+typedef struct {
+    const uint8_t *packed;
+    int64_t n;
+    int64_t k;
+    float scale;
+} bitnet_tw;
+
+#define BITNET_MAX_K 65536
+/* Largest number of tokens the decode (GEMV) path takes in one pass; larger M
+ * runs through the tensor-core GEMM path. */
+#define BITNET_GEMV_MAX_M 8
+/* Largest number of layers one bitnet_linear_stack call takes. */
+#define BITNET_STACK_MAX 256
+
+/* Library version as 10000*major + 100*minor + patch. */
+BITNET_API int bitnet_version(void);
+
+/* Text of a status code (static storage). */
+BITNET_API const char *bitnet_status_str(bitnet_status s);
+
+/* Detail of the last error returned on the calling thread (static storage,
+ * overwritten by the next failing call). */
+BITNET_API const char *bitnet_last_error(void);
+
+/* Map a *d_flags word read back from the device to a status
+ * (TIMEOUT > NONFINITE > NOT_TERNARY > OK in priority). */
+BITNET_API bitnet_status bitnet_status_from_flags(int32_t flags);
+
+/* Bytes of a packed [n, k] tensor: n * 32 * ceil(k/128); 0 on bad sizes. */
+BITNET_API size_t bitnet_packed_bytes(int64_t n, int64_t k);
+
+/* Padded int8 row width 128 * ceil(k/128); 0 on bad sizes. */
+BITNET_API int64_t bitnet_kpad(int64_t k);
+
+/*
+ * Pack int8 ternary weights into the 2-bit format (the I2_S weight storage of
+ * the technical report §2.2.2; 128-element blocks per the blog post's second
+ * postscript).
+ *   w      device, int8 [n, k], values in {-1, 0, +1}
+ *   packed device, [n, 32*ceil(k/128)] bytes, 16-byte aligned; fully written
+ * A value outside {-1,0,+1} is stored as weight 0 and raises
+ * BITNET_FLAG_NOT_TERNARY in *d_flags.  Load-time operation.
+ */
+BITNET_API bitnet_status bitnet_pack_ternary(const int8_t *w, int64_t n, int64_t k,
+                                  uint8_t *packed, int32_t *d_flags, void *stream);
+
+/* Inverse of bitnet_pack_ternary (test and inspection aid):
+ *   packed device [n, 32*ceil(k/128)] -> w device int8 [n, k]. */
+BITNET_API bitnet_status bitnet_unpack_ternary(const uint8_t *packed, int64_t n, int64_t k,
+                                    int8_t *w, void *stream);
+
+/*
+ * Per-token int8 activation quantiser (technical report §2.2.2: activations
+ * quantised to INT8 per token at run time; absmax/127 rule above).
+ *   x         device fp32 [m, k], 16-byte aligned
+ *   xq        device int8 [m, kpad], kpad = bitnet_kpad(k), pads written as 0
+ *   act_scale device fp32 [m]
+ * Non-finite rows raise BITNET_FLAG_NONFINITE.
+ */
+BITNET_API bitnet_status bitnet_quant_act(const float *x, int64_t m, int64_t k, int8_t *xq,
+                               float *act_scale, int32_t *d_flags, void *stream);
+
+/* Workspace bytes bitnet_linear needs for m tokens of width k: 0 when
+ * m <= BITNET_GEMV_MAX_M (the quantiser is fused into the GEMV), otherwise
+ * room for the int8 activations and their scales. */
+BITNET_API size_t bitnet_linear_workspace_bytes(int64_t m, int64_t k);
+
+/*
+ * One ternary linear layer y = dequant(quant(x) W^T) (technical report
+ * §2.2.2, §2.4.2 and Figure 4: unpack the 2-bit weights to int8, multiply-add
+ * into int32, per-token and per-tensor scales in fp32).
+ *   x         device fp32 [m, w->k], 16-byte aligned, m >= 1
+ *   w         host pointer to the weight descriptor
+ *   y         device fp32 [m, w->n]
+ *   acc_out   device int32 [m, w->n] or NULL: the exact integer sums
+ *   workspace device, 256-byte aligned, >= bitnet_linear_workspace_bytes(m,k)
+ *             bytes (may be NULL when that is 0); owned by the caller, must not
+ *             be used by another call until this one has completed on `stream`
+ * m <= 8 runs the fused quantiser + streaming GEMV; larger m quantises into
+ * the workspace and runs the tensor-core GEMM.
+ */
+BITNET_API bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_tw *w, float *y,
+                            int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                            int32_t *d_flags, void *stream);
+
+/*
+ * The same layer on activations already quantised by bitnet_quant_act
+ * (prefill on pre-quantised A).
+ *   xq        device int8 [m, bitnet_kpad(w->k)], 16-byte aligned, pads 0
+ *   act_scale device fp32 [m]
+ */
+BITNET_API bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t m,
+                              const bitnet_tw *w, float *y, int32_t *acc_out,
+                              int32_t *d_flags, void *stream);
+
+/*
+ * A sequence of `count` independent ternary linear layers sharing the token
+ * count m, run in one launch (the decoder's linears back to back: each
+ * token reads every layer's weights once, technical report §2.2.2 and §3.2,
+ * Figure 6 decode).
+ *   x[i]      device fp32 [m, w[i].k]; the same pointer may feed several
+ *             layers (it is quantised once per use within a CTA)
+ *   w         host array of `count` descriptors
+ *   y[i]      device fp32 [m, w[i].n]; outputs must not overlap any input
+ *   acc_out   NULL, or host array of `count` device int32 [m, w[i].n]
+ *             pointers (entries may be NULL)
+ * 1 <= count <= BITNET_STACK_MAX.  m > BITNET_GEMV_MAX_M is processed in
+ * slices of at most BITNET_GEMV_MAX_M tokens.
+ */
+BITNET_API bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet_tw *w,
+                                  int64_t count, float *const *y, int32_t *const *acc_out,
+                                  int32_t *d_flags, void *stream);
+
+/* Test aid: bound, in SM clock cycles, on every device-side wait (0 = the
+ * built-in bound of about 2^31 cycles).  A wait that runs past it makes the
+ * kernel raise BITNET_FLAG_TIMEOUT and return instead of hanging.
+ * Process-wide; affects launches made after the call. */
+BITNET_API bitnet_status bitnet_debug_set_wait_limit(uint64_t cycles);
+
+/* Test aid: when on, the GEMV kernels of later launches first wait on a
+ * barrier that nothing ever completes, so that the bounded wait expires; they
+ * raise BITNET_FLAG_TIMEOUT and return without writing outputs.  Used to test
+ * the timeout path without faulting or hanging a GPU.  Process-wide. */
+BITNET_API bitnet_status bitnet_debug_force_stall(int on);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITNET_H */

@@ -1,0 +1,144 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of the library.
+//
+// Only inline PTX for the primitives the kernels use: mbarriers, 1-D bulk
+// (TMA) copies global->shared, dp4a, bounded waits.  Every wait is bounded by
+// a clock limit; on expiry the caller raises BITNET_FLAG_TIMEOUT and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/bitnet.h"
+
+// The library is written for B200 only.  Building the device code for any
+// other architecture is an error, not a silent empty kernel.
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
+#error "bitnet kernels target sm_100a (B200) only: build with -gencode arch=compute_100a,code=sm_100a"
+#endif
+
+namespace bitnet {
+
+constexpr uint64_t kDefaultWaitLimit = (1ull << 31);   // ~1 s at 2 GHz
+constexpr uint64_t kDrainWaitLimit = (1ull << 31);
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void raise_flag(int32_t *flags, int32_t bit)
+{
+    if (flags) atomicOr(flags, bit);
+}
+
+// ------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of parity `parity` to complete; false if `limit` SM
+// cycles pass first.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = clock64();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// ------------------------------------------------------------ bulk copies
+
+// 1-D bulk asynchronous copy global -> shared (TMA engine), completion
+// counted in bytes on `bar`.  dst, src 16-byte aligned; bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// ----------------------------------------------------------- arithmetic
+
+// Four-way byte dot product: unsigned bytes of a times signed bytes of b,
+// accumulated into c (the u8 x s8 multiply-add of the unpack-and-madd
+// formulation).
+__device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c)
+{
+    int32_t d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int32_t warp_sum(int32_t v)
+{
+    return __reduce_add_sync(0xffffffffu, v);
+}
+
+// Per-token activation quantiser of one element given inv = 127/amax
+// (round half to even, clamp to +-127, zero stays zero).
+__device__ __forceinline__ int32_t quant_one(float x, float inv)
+{
+    if (x == 0.0f) return 0;
+    float v = __fmul_rn(x, inv);
+    v = fminf(fmaxf(v, -127.0f), 127.0f);
+    return __float2int_rn(v);
+}
+
+__device__ __forceinline__ uint32_t pack4(int32_t a, int32_t b, int32_t c, int32_t d)
+{
+    return (uint32_t(a) & 0xffu) | ((uint32_t(b) & 0xffu) << 8) | ((uint32_t(c) & 0xffu) << 16) |
+           ((uint32_t(d) & 0xffu) << 24);
+}
+
+}  // namespace bitnet

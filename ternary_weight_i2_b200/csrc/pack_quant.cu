@@ -1,0 +1,154 @@
+// pack_quant.cu -- load-time pack/unpack of the 2-bit ternary format and the
+// standalone per-token int8 activation quantiser (prefill input).
+//
+// Format ("VibeVoice-ASR-BitNet Technical Report", §2.2.2: ternary weights in
+// 2 bits; 128-element groups per the ARM debugging blog post, second
+// postscript): element k = 128j + 32g + b of a row sits in byte 32j + b, bits
+// [2g, 2g+1], as code w + 1; tail positions hold code 1 (weight 0).
+#include "common.cuh"
+
+namespace bitnet {
+
+// One thread per packed byte: gathers the four elements 128j + 32g + b.
+__global__ void pack_kernel(const int8_t *__restrict__ w, int64_t n, int64_t k, int64_t kb,
+                            uint8_t *__restrict__ packed, int32_t *flags)
+{
+    const int64_t rowb = 32 * kb;
+    const int64_t total = n * rowb;
+    bool bad = false;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+         idx += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / rowb, byte = idx - r * rowb;
+        const int64_t j = byte >> 5, b = byte & 31;
+        uint32_t out = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int64_t kk = 128 * j + 32 * g + b;
+            uint32_t code = 1;
+            if (kk < k) {
+                const int v = w[r * k + kk];
+                if (v >= -1 && v <= 1) code = uint32_t(v + 1);
+                else bad = true;
+            }
+            out |= code << (2 * g);
+        }
+        packed[idx] = uint8_t(out);
+    }
+    const unsigned mask = __ballot_sync(0xffffffffu, bad);
+    if (mask != 0u && (threadIdx.x & 31) == unsigned(__ffs(mask) - 1)) raise_flag(flags, BITNET_FLAG_NOT_TERNARY);
+}
+
+__global__ void unpack_kernel(const uint8_t *__restrict__ packed, int64_t n, int64_t k, int64_t kb,
+                              int8_t *__restrict__ w)
+{
+    const int64_t rowb = 32 * kb;
+    const int64_t total = n * rowb;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+         idx += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / rowb, byte = idx - r * rowb;
+        const int64_t j = byte >> 5, b = byte & 31;
+        const uint32_t v = packed[idx];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int64_t kk = 128 * j + 32 * g + b;
+            if (kk < k) w[r * k + kk] = int8_t(int((v >> (2 * g)) & 3u) - 1);
+        }
+    }
+}
+
+// Per-token quantiser: one CTA per row.  Pass 1 finds absmax (and whether the
+// row is finite), pass 2 writes rint(x * 127/amax) as int8 in natural order,
+// four codes per 32-bit store, pads zero.
+template <int NT>
+__global__ void __launch_bounds__(NT) quant_kernel(const float *__restrict__ x, int64_t m, int64_t k,
+                                                   int64_t kpad, int8_t *__restrict__ xq,
+                                                   float *__restrict__ scale, int32_t *flags)
+{
+    __shared__ float s_max[NT / 32];
+    __shared__ int s_bad[NT / 32];
+    const int64_t r = blockIdx.x;
+    const float *row = x + r * k;
+    const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15) == 0);
+    const int64_t nw = kpad / 4;
+    float a = 0.f;
+    bool bad = false;
+    auto load = [&](int64_t wi) -> float4 {
+        const int64_t k0 = 4 * wi;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (vec && k0 + 3 < k) {
+            v = __ldg(reinterpret_cast<const float4 *>(row + k0));
+        } else {
+            if (k0 + 0 < k) v.x = __ldg(row + k0 + 0);
+            if (k0 + 1 < k) v.y = __ldg(row + k0 + 1);
+            if (k0 + 2 < k) v.z = __ldg(row + k0 + 2);
+            if (k0 + 3 < k) v.w = __ldg(row + k0 + 3);
+        }
+        return v;
+    };
+    for (int64_t wi = threadIdx.x; wi < nw; wi += NT) {
+        const float4 v = load(wi);
+        const bool fin = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+        if (!fin) bad = true;
+        else a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    a = warp_max(a);
+    const bool wbad = __any_sync(0xffffffffu, bad);
+    if ((threadIdx.x & 31) == 0) {
+        s_max[threadIdx.x >> 5] = a;
+        s_bad[threadIdx.x >> 5] = wbad ? 1 : 0;
+    }
+    __syncthreads();
+    float amax = 0.f;
+    int anybad = 0;
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) {
+        amax = fmaxf(amax, s_max[i]);
+        anybad |= s_bad[i];
+    }
+    const bool zero = anybad || amax == 0.f;
+    const float inv = zero ? 0.f : __fdiv_rn(127.0f, amax);
+    uint32_t *out = reinterpret_cast<uint32_t *>(xq + r * kpad);
+    for (int64_t wi = threadIdx.x; wi < nw; wi += NT) {
+        uint32_t word = 0;
+        if (!zero) {
+            const float4 v = load(wi);
+            word = pack4(quant_one(v.x, inv), quant_one(v.y, inv), quant_one(v.z, inv), quant_one(v.w, inv));
+        }
+        out[wi] = word;
+    }
+    if (threadIdx.x == 0) {
+        scale[r] = zero ? 0.f : __fdiv_rn(amax, 127.0f);
+        if (anybad) raise_flag(flags, BITNET_FLAG_NONFINITE);
+    }
+}
+
+static int grid_for(int64_t work, int threads)
+{
+    int64_t g = (work + threads - 1) / threads;
+    if (g > 148 * 32) g = 148 * 32;
+    return int(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_pack(const int8_t *w, int64_t n, int64_t k, uint8_t *packed, int32_t *flags, cudaStream_t st)
+{
+    const int64_t kb = (k + 127) / 128;
+    pack_kernel<<<grid_for(n * 32 * kb, 256), 256, 0, st>>>(w, n, k, kb, packed, flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const uint8_t *packed, int64_t n, int64_t k, int8_t *w, cudaStream_t st)
+{
+    const int64_t kb = (k + 127) / 128;
+    unpack_kernel<<<grid_for(n * 32 * kb, 256), 256, 0, st>>>(packed, n, k, kb, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float *scale, int32_t *flags,
+                         cudaStream_t st)
+{
+    const int64_t kpad = 128 * ((k + 127) / 128);
+    quant_kernel<256><<<unsigned(m), 256, 0, st>>>(x, m, k, kpad, xq, scale, flags);
+    return cudaGetLastError();
+}
+
+}  // namespace bitnet
