@@ -49,6 +49,10 @@ def _args():
     ap.add_argument("--no-sweep", action="store_true", help="skip the M = 2, 4, 8 lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--soak", type=float, default=0.5,
+                    help="seconds of untimed launches before timing (clock sampling window)")
+    ap.add_argument("--layers", type=int, default=28,
+                    help="decoder layers in the stack (28 = the benchmark; fewer only for profiling captures)")
     return ap.parse_args()
 
 
@@ -85,62 +89,60 @@ def _ncu_traffic(m):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons polled through NVML every
+    ~2 ms from a background thread while the timed region runs."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.reasons = set()
+        self.stop_evt = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of numbers
+            self.err = str(e)
+
+    def _poll(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+        if self.ok:
+            self.t = threading.Thread(target=self._poll, daemon=True)
             self.t.start()
-        except Exception:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable: " + self.err]}
+        self.stop_evt.set()
         self.t.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ GPU arm
 
-def build_stack(m, dev):
+def build_stack(m, dev, layers=28):
     """Pack the 28 layers on the GPU; return descriptors, the contiguous input
     and output buffers and their per-layer views."""
     import torch
@@ -148,7 +150,7 @@ def build_stack(m, dev):
     from ternary_weight_i2_b200 import synth
 
     packed, tws = [], []
-    for L in range(synth.NUM_LAYERS):
+    for L in range(layers):
         for (name, n, k), (w, s) in zip(synth.LAYER_SHAPES, synth.layer_weights(L, 3)):
             wt = torch.from_numpy(w).to(dev)
             pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
@@ -159,18 +161,18 @@ def build_stack(m, dev):
             tws.append(tw2.make_tw(pk, n, k, s))
     torch.cuda.synchronize()
     # all distinct inputs in one buffer, all outputs in another
-    in_sizes = [m * k for _ in range(synth.NUM_LAYERS) for k in synth.LAYER_INPUT_K]
-    out_sizes = [m * n for _ in range(synth.NUM_LAYERS) for (_, n, _) in synth.LAYER_SHAPES]
+    in_sizes = [m * k for _ in range(layers) for k in synth.LAYER_INPUT_K]
+    out_sizes = [m * n for _ in range(layers) for (_, n, _) in synth.LAYER_SHAPES]
     x_host = np.empty(sum(in_sizes), np.float32)
     off = 0
-    for L in range(synth.NUM_LAYERS):
+    for L in range(layers):
         for a in synth.layer_inputs(L, m, 3):
             x_host[off:off + a.size] = a.ravel()
             off += a.size
     x_dev = torch.from_numpy(x_host).to(dev)
     y_dev = torch.empty(sum(out_sizes), dtype=torch.float32, device=dev)
     xs, ys, off, yoff = [], [], 0, 0
-    for L in range(synth.NUM_LAYERS):
+    for L in range(layers):
         views = []
         for k in synth.LAYER_INPUT_K:
             views.append(x_dev[off:off + m * k].view(m, k))
@@ -237,7 +239,8 @@ def run_gpu(args):
     tw2.load()
 
     m = args.m
-    packed, tws, xs, ys, x_host, x_dev, y_dev = build_stack(m, dev)
+    packed, tws, xs, ys, x_host, x_dev, y_dev = build_stack(m, dev, args.layers)
+    stack_bytes = sum(int(p.numel()) for p in packed)
     flags = torch.zeros(1, dtype=torch.int32, device=dev)
     call = tw2.StackCall(xs, tws, ys)
     stream = torch.cuda.current_stream()
@@ -250,6 +253,8 @@ def run_gpu(args):
         call(flags=flags)
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(local)
+    for _ in range(int(args.soak / 1e-4)):   # untimed soak of the same launch before timing
+        graph.replay()
     clocks.start()
     total_ms, per = time_device(graph.replay, args.steps, args.warmup, stream)
     clk = clocks.stop()
@@ -278,25 +283,29 @@ def run_gpu(args):
                "h2d_bytes_per_step": int(x_host.nbytes), "d2h_bytes_per_step": int(y_dev.numel() * 4)}
 
     peak, peak_kind, peaks = _peaks()
-    achieved = STACK_BYTES / (kern_ms * 1e-3) / 1e9
+    achieved = stack_bytes / (kern_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": _ncu_traffic(m),
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "kernel": "gemv_stack_kernel", "kernel_ms": round(kern_ms, 5),
-                "algorithmic_bytes": STACK_BYTES}
+                "algorithmic_bytes": stack_bytes}
 
     sweep = {}
     if not args.no_sweep and m == 1:
         for ms in (2, 4, 8):
-            _, twsm, xsm, ysm, _, _, _ = build_stack_views(ms, dev, tws)
+            _, twsm, xsm, ysm, _, _, _ = build_stack_views(ms, dev, tws, args.layers)
             c2 = tw2.StackCall(xsm, twsm, ysm)
             c2(flags=flags)
-            t2, per2 = time_device(lambda: c2(flags=flags), 50, 5, stream)
+            torch.cuda.synchronize()
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                c2(flags=flags)
+            t2, per2 = time_device(g2.replay, 50, 5, stream)
             t2 = _max_over_ranks(t2)
             k2 = _max_over_ranks(statistics.mean(per2))
             sweep[str(ms)] = {"tokens_per_s": round(world * ms / (t2 / 50 * 1e-3), 1),
-                              "weight_gbs": round(STACK_BYTES / (k2 * 1e-3) / 1e9, 1)}
+                              "weight_gbs": round(stack_bytes / (k2 * 1e-3) / 1e9, 1)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -308,13 +317,14 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
             "data": "synthetic (seeded ternary weights and fp32 activations, BASELINE shapes)",
-            "config": {"workload": "28-layer ternary linear stack, 196 layers, M=%d decode" % m,
-                       "tokens_per_step_per_gpu": m, "layers": 196,
-                       "packed_weight_bytes": STACK_BYTES,
+            "config": {"workload": "%d-layer ternary linear stack, %d layers, M=%d decode"
+                                   % (args.layers, 7 * args.layers, m),
+                       "tokens_per_step_per_gpu": m, "layers": 7 * args.layers,
+                       "packed_weight_bytes": stack_bytes,
                        "l2": "weights 327.5 MB > 126 MB L2 (no flush needed)",
                        "parallelism": "replicas" if world > 1 else "single GPU",
                        "timing": "CUDA graph replay of one bitnet_linear_stack launch per step"},
-            "weight_gbs": round(STACK_BYTES * world / (ms_step * 1e-3) / 1e9, 1),
+            "weight_gbs": round(stack_bytes * world / (ms_step * 1e-3) / 1e9, 1),
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -327,12 +337,12 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def build_stack_views(m, dev, tws):
+def build_stack_views(m, dev, tws, layers=28):
     """Inputs/outputs for another token count, reusing the packed weights."""
     import torch
     from ternary_weight_i2_b200 import synth
     xs, ys = [], []
-    for L in range(synth.NUM_LAYERS):
+    for L in range(layers):
         views = [torch.from_numpy(a).to(dev) for a in synth.layer_inputs(L, m, 3)]
         for (_, n, _), j in zip(synth.LAYER_SHAPES, synth.LAYER_INPUT_OF):
             xs.append(views[j])

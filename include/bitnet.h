@@ -15,6 +15,14 @@
  * - Pointers named d_* or documented "device" point to CUDA device memory of
  *   the current device; the caller owns every buffer.  Functions that take a
  *   workspace never allocate; no function allocates device memory per call.
+ *   The GEMV path (bitnet_linear with m <= 8, bitnet_linear_q with m <= 8,
+ *   bitnet_linear_stack) streams each weight tensor through a TMA tensor map
+ *   that the library encodes the first time it meets that tensor (same
+ *   packed pointer, n and k) and keeps in a per-device cache (128 bytes of
+ *   device memory per tensor, allocated 128 KB at a time, until
+ *   bitnet_release_device_cache() or exit).  That first call allocates and
+ *   copies synchronously, so it must not be made under CUDA stream capture;
+ *   later calls with the same tensors only look the maps up.
  * - `stream` is a cudaStream_t (NULL = legacy default stream).  All GPU work is
  *   enqueued on it and the functions return without synchronising.
  * - Errors found on the host (bad argument, misaligned pointer, device that is
@@ -196,6 +204,10 @@ BITNET_API bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, c
                                   int64_t count, float *const *y, int32_t *const *acc_out,
                                   int32_t *d_flags, void *stream);
 
+/* Free the current device's tensor-map cache (waits for the device to be
+ * idle first).  Later calls rebuild entries as needed. */
+BITNET_API bitnet_status bitnet_release_device_cache(void);
+
 /* Test aid: bound, in SM clock cycles, on every device-side wait (0 = the
  * built-in bound of about 2^31 cycles).  A wait that runs past it makes the
  * kernel raise BITNET_FLAG_TIMEOUT and return instead of hanging.
@@ -207,6 +219,14 @@ BITNET_API bitnet_status bitnet_debug_set_wait_limit(uint64_t cycles);
  * raise BITNET_FLAG_TIMEOUT and return without writing outputs.  Used to test
  * the timeout path without faulting or hanging a GPU.  Process-wide. */
 BITNET_API bitnet_status bitnet_debug_force_stall(int on);
+
+/* Profiling aid: when d_trace (device memory) is not NULL, GEMV launches made
+ * after the call write, per CTA c and warp w of the launch, 8 uint64
+ * %globaltimer stamps (ns) at d_trace[(c*warps + w)*8 + e]: e = 0 set-up done,
+ * 1 first weight copies issued, 2 activations quantised, 3 first chunk landed,
+ * 4 last chunk consumed (other slots unused).  The buffer must hold
+ * 8 * warps * CTAs entries (at most 8 * 16 * 160).  NULL turns it off. */
+BITNET_API bitnet_status bitnet_debug_set_trace(void *d_trace);
 
 #ifdef __cplusplus
 }

@@ -51,6 +51,8 @@ _SIGNATURES = {
     "bitnet_linear_stack": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
+    "bitnet_debug_set_trace": ([_P], C.c_int),
+    "bitnet_release_device_cache": ([], C.c_int),
 }
 
 _lib = None
@@ -123,8 +125,18 @@ def linear_workspace_bytes(m: int, k: int) -> int:
     return int(load().bitnet_linear_workspace_bytes(m, k))
 
 
+def release_device_cache() -> None:
+    _check(load().bitnet_release_device_cache(), "bitnet_release_device_cache")
+
+
 def set_wait_limit(cycles: int) -> None:
     _check(load().bitnet_debug_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+def set_trace(buf) -> None:
+    """Profiling aid: per-warp phase timestamps of later GEMV launches go to
+    ``buf`` (a uint64/int64 device tensor of 8*16*160 entries), None to stop."""
+    _check(load().bitnet_debug_set_trace(_ptr(buf)), "set_trace")
 
 
 def force_stall(on: bool) -> None:

@@ -1,16 +1,21 @@
 // capi.cu -- the C ABI declared in include/bitnet.h: argument checks, the
 // device check, work partitioning for the streaming GEMV, and dispatch.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "common.cuh"
 #include "gemv.cuh"
 
 namespace bitnet {
-cudaError_t launch_gemv(const GemvParams &p, int nw, cudaStream_t st);
+cudaError_t launch_gemv(const GemvParams &p, int variant, cudaStream_t st);
 cudaError_t launch_pack(const int8_t *w, int64_t n, int64_t k, uint8_t *packed, int32_t *flags, cudaStream_t st);
 cudaError_t launch_unpack(const uint8_t *packed, int64_t n, int64_t k, int8_t *w, cudaStream_t st);
 cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float *scale, int32_t *flags,
@@ -27,6 +32,7 @@ namespace {
 thread_local char g_err[512] = "";
 uint64_t g_wait_limit = 0;   // 0: built-in bound
 int g_force_stall = 0;       // test aid: kernels wait on a barrier nobody arrives at
+uint64_t *g_trace = nullptr; // optional device buffer for per-warp phase timestamps
 
 bitnet_status fail(bitnet_status s, const char *fmt, ...)
 {
@@ -48,6 +54,7 @@ int64_t blocks_of(int64_t k) { return (k + 127) / 128; }
 
 struct DevInfo {
     int sm_count = 0;
+    int ordinal = 0;
     bool ok = false;
 };
 
@@ -76,6 +83,7 @@ bitnet_status check_device(DevInfo *info)
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         cache[dev].sm_count = n;
+        cache[dev].ordinal = dev;
         cache[dev].ok = true;
         cached[dev] = true;
     }
@@ -97,6 +105,113 @@ bitnet_status check_tw(const bitnet_tw &w, int64_t i)
 
 uint64_t wait_limit() { return g_wait_limit ? g_wait_limit : kDefaultWaitLimit; }
 
+// ------------------------------------------------------- tensor-map cache
+//
+// The GEMV streams each packed weight matrix through a 2-D tiled TMA tensor
+// map (uint8, dims {32*kb bytes, n rows}, box {128, 32}, 128-byte swizzle,
+// zero fill out of bounds).  A map depends only on (address, n, kb), so maps
+// are encoded once on the host and kept, per device, in device memory that
+// lives until bitnet_release_device_cache() or process exit.  The first call
+// that meets a new weight tensor allocates and copies (it must not run under
+// stream capture); later calls only look the map up.
+
+struct TmapKey {
+    const void *p;
+    int64_t n, kb;
+    bool operator==(const TmapKey &o) const { return p == o.p && n == o.n && kb == o.kb; }
+};
+struct TmapKeyHash {
+    size_t operator()(const TmapKey &k) const
+    {
+        return std::hash<const void *>()(k.p) ^ (std::hash<int64_t>()(k.n) * 31u) ^ (std::hash<int64_t>()(k.kb) * 131u);
+    }
+};
+constexpr int kTmapChunk = 1024;
+struct TmapChunk {
+    CUtensorMap *dev = nullptr;
+    CUtensorMap *host = nullptr;   // pinned mirror, each entry written once
+    int used = 0;
+};
+struct DeviceTmaps {
+    std::unordered_map<TmapKey, const CUtensorMap *, TmapKeyHash> index;
+    std::vector<TmapChunk> chunks;
+};
+std::mutex g_tmap_mu;
+DeviceTmaps g_tmaps[64];
+uint64_t g_tmap_generation = 1;   // bumped when a cache is released
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+bitnet_status encode_weight_map(CUtensorMap *out, const void *packed, int64_t n, int64_t kb)
+{
+    auto fn = encode_fn();
+    if (!fn) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[2] = {cuuint64_t(32 * kb), cuuint64_t(n)};
+    const cuuint64_t strides[1] = {cuuint64_t(32 * kb)};
+    const cuuint32_t box[2] = {128u, cuuint32_t(kTileRows)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(packed), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+    return BITNET_OK;
+}
+
+// Device tensor maps of `count` weight tensors; new ones are encoded and
+// copied in one batch per chunk.
+bitnet_status weight_maps(int dev, const bitnet_tw *const *w, int count, const void **out)
+{
+    std::lock_guard<std::mutex> lock(g_tmap_mu);
+    DeviceTmaps &D = g_tmaps[dev];
+    std::vector<std::pair<int, int>> fresh;   // (chunk, first new entry)
+    for (int i = 0; i < count; ++i) {
+        const TmapKey key{w[i]->packed, w[i]->n, blocks_of(w[i]->k)};
+        auto it = D.index.find(key);
+        if (it != D.index.end()) {
+            out[i] = it->second;
+            continue;
+        }
+        if (D.chunks.empty() || D.chunks.back().used == kTmapChunk) {
+            TmapChunk c;
+            cudaError_t e = cudaMalloc(&c.dev, kTmapChunk * sizeof(CUtensorMap));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(tensor-map cache)");
+            e = cudaMallocHost(&c.host, kTmapChunk * sizeof(CUtensorMap));
+            if (e != cudaSuccess) {
+                cudaFree(c.dev);
+                return cuda_fail(e, "cudaMallocHost(tensor-map cache)");
+            }
+            D.chunks.push_back(c);
+        }
+        TmapChunk &c = D.chunks.back();
+        const int ci = int(D.chunks.size()) - 1;
+        if (fresh.empty() || fresh.back().first != ci) fresh.emplace_back(ci, c.used);
+        bitnet_status s = encode_weight_map(&c.host[c.used], key.p, key.n, key.kb);
+        if (s != BITNET_OK) return s;
+        const CUtensorMap *d = c.dev + c.used;
+        ++c.used;
+        D.index.emplace(key, d);
+        out[i] = d;
+    }
+    for (auto &f : fresh) {
+        TmapChunk &c = D.chunks[f.first];
+        cudaError_t e = cudaMemcpy(c.dev + f.second, c.host + f.second, size_t(c.used - f.second) * sizeof(CUtensorMap),
+                                   cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-map upload");
+    }
+    return BITNET_OK;
+}
+
 // ---------------------------------------------------------------- GEMV plan
 
 struct LayerReq {
@@ -107,23 +222,89 @@ struct LayerReq {
     int32_t *acc;
 };
 
-int nw_for(int m)
+// Kernel variant for m tokens whose activation area holds an input of
+// max_kpad columns; BITNET_TEST_GEMV_VARIANT (tuning aid) forces one.
+int pick_variant(int m, int64_t max_kpad)
 {
-    if (m <= 1) return 8;
-    if (m <= 5) return 6;
-    return 4;
+    static const int pref[9][4] = {{-1}, {0, 1, 3, -1}, {0, 2, 3, -1}, {2, 3, -1}, {2, 3, -1}, {2, 3, -1},
+                                   {3, -1}, {3, -1}, {3, -1}};
+    if (const char *f = getenv("BITNET_TEST_GEMV_VARIANT")) {
+        const int v = atoi(f);
+        if (v >= 0 && v < kNumVariants && m <= kVariantMaxM[v] &&
+            int64_t(m) * max_kpad <= x_cap(kVariants[v].nw, kVariants[v].boxes))
+            return v;
+    }
+    for (int i = 0; i < 4 && pref[m][i] >= 0; ++i) {
+        const int v = pref[m][i];
+        if (int64_t(m) * max_kpad <= x_cap(kVariants[v].nw, kVariants[v].boxes)) return v;
+    }
+    return -1;
 }
 
-// Split the layers' 32-row tiles into contiguous byte-balanced ranges (one CTA
-// each) under the per-CTA limits: distinct inputs, segments, and the shared
-// memory that holds the quantised activations.
+// Plans of recent launches, reused when a call repeats its arguments exactly
+// (decode loops call the same stack with the same buffers every step).
+struct PlanKey {
+    std::vector<LayerReq> layers;
+    int m = 0;
+    bool prequant = false;
+    int32_t *flags = nullptr;
+    int ordinal = -1;
+    uint64_t generation = 0, wait_limit = 0;
+    int force_stall = 0;
+    uint64_t *trace = nullptr;
+    bool matches(const std::vector<LayerReq> &L, int m_, bool pq, int32_t *fl, int dev, uint64_t gen) const
+    {
+        if (m != m_ || prequant != pq || flags != fl || ordinal != dev || generation != gen ||
+            wait_limit != g_wait_limit || force_stall != g_force_stall ||
+            trace != g_trace || layers.size() != L.size())
+            return false;
+        return std::memcmp(layers.data(), L.data(), L.size() * sizeof(LayerReq)) == 0;
+    }
+};
+struct CachedPlan {
+    PlanKey key;
+    GemvParams params;
+    int variant = -1;
+};
+constexpr int kPlanCacheSize = 8;
+thread_local std::vector<CachedPlan> g_plans;
+thread_local int g_plan_next = 0;
+
+// Split the layers' 32-row tiles into contiguous ranges, one CTA each: tile
+// t goes to range floor((bytes before t + half of t) * G / total), so every
+// range holds within half a tile of total/G bytes (G = SM count).  A range is
+// split further when it would exceed a per-CTA limit (distinct inputs,
+// segments, shared memory for the quantised activations).
 bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequant, int32_t *flags,
                               cudaStream_t st, const DevInfo &dev)
 {
-    static thread_local GemvParams p;   // host staging of the kernel parameter block
+    uint64_t gen;
+    {
+        std::lock_guard<std::mutex> lock(g_tmap_mu);
+        gen = g_tmap_generation;
+    }
+    for (const CachedPlan &c : g_plans)
+        if (c.key.matches(L, m, prequant, flags, dev.ordinal, gen)) {
+            cudaError_t e = launch_gemv(c.params, c.variant, st);
+            return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
+        }
+    if (int(g_plans.size()) < kPlanCacheSize) g_plans.emplace_back();
+    CachedPlan &slot_plan = g_plans[g_plan_next];
+    g_plan_next = (g_plan_next + 1) % kPlanCacheSize;
+    slot_plan.variant = -1;   // invalid until the plan below succeeds
+    GemvParams &p = slot_plan.params;
     static thread_local std::vector<int> input_of;
     const int count = int(L.size());
-    // distinct inputs: same pointer and same width
+    {
+        static thread_local std::vector<const bitnet_tw *> wp;
+        static thread_local std::vector<const void *> maps;
+        wp.resize(count);
+        maps.resize(count);
+        for (int i = 0; i < count; ++i) wp[i] = &L[i].w;
+        bitnet_status s = weight_maps(dev.ordinal, wp.data(), count, maps.data());
+        if (s != BITNET_OK) return s;
+        for (int i = 0; i < count; ++i) p.lin[i].tmap = maps[i];
+    }
     int ninp = 0;
     input_of.assign(count, -1);
     int64_t max_kpad = 0;
@@ -145,7 +326,6 @@ bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequa
         input_of[i] = found;
         const int64_t kp = 128 * blocks_of(L[i].w.k);
         if (kp > max_kpad) max_kpad = kp;
-        p.lin[i].packed = L[i].w.packed;
         p.lin[i].y = L[i].y;
         p.lin[i].acc = L[i].acc;
         p.lin[i].n = int32_t(L[i].w.n);
@@ -153,60 +333,60 @@ bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequa
         p.lin[i].scale = L[i].w.scale;
         p.lin[i].input = found;
     }
-    int nw = nw_for(m);
-    if (int64_t(m) * max_kpad > gemv_x_cap(nw)) nw = 4;
-    if (int64_t(m) * max_kpad > gemv_x_cap(nw))
+    const int variant = pick_variant(m, max_kpad);
+    if (variant < 0)
         return fail(BITNET_ERR_INVALID_ARG, "m=%d x kpad=%lld exceeds the GEMV activation area", m,
                     (long long)max_kpad);
-    const int64_t xcap = gemv_x_cap(nw);
+    const int64_t xcap = x_cap(kVariants[variant].nw, kVariants[variant].boxes);
 
     int64_t total = 0;
     for (int i = 0; i < count; ++i) total += L[i].w.n * 32 * blocks_of(L[i].w.k);
-    int64_t target = (total + dev.sm_count - 1) / dev.sm_count;
-    for (int attempt = 0; attempt < 8; ++attempt, target += target / 2 + 1) {
-        int nr = 0, ns = 0;
-        bool open = false, overflow = false;
-        int64_t cur_bytes = 0, cur_x = 0, xmax = 0;
-        auto open_range = [&]() -> bool {
-            if (nr == kMaxRanges) return false;
-            GemvRange &r = p.rng[nr];
-            r.seg0 = int16_t(ns);
-            r.nseg = 0;
-            r.nin = 0;
-            cur_bytes = 0;
-            cur_x = 0;
-            open = true;
-            return true;
-        };
-        auto close_range = [&]() {
-            if (open && p.rng[nr].nseg > 0) {
-                xmax = cur_x > xmax ? cur_x : xmax;
-                ++nr;
-            }
-            open = false;
-        };
-        for (int i = 0; i < count && !overflow; ++i) {
-            const int64_t rowb = 32 * blocks_of(L[i].w.k);
-            const int64_t tiles = (L[i].w.n + kTileRows - 1) / kTileRows;
-            const int64_t tb = kTileRows * rowb;
-            const int64_t xin = int64_t(m) * 128 * blocks_of(L[i].w.k);
-            int64_t t = 0;
-            while (t < tiles) {
-                if (!open && !open_range()) {
-                    overflow = true;
-                    break;
+    const int64_t G = dev.sm_count;
+
+    int nr = 0, ns = 0;
+    int64_t cur_x = 0, xmax = 0, cum = 0;
+    int cur_target = -1;   // balanced-range index the open range belongs to
+    bool open = false;
+    auto close_range = [&]() {
+        if (open && p.rng[nr].nseg > 0) {
+            xmax = cur_x > xmax ? cur_x : xmax;
+            ++nr;
+        }
+        open = false;
+    };
+    for (int i = 0; i < count; ++i) {
+        const int64_t rowb = 32 * blocks_of(L[i].w.k);
+        const int64_t tiles = (L[i].w.n + kTileRows - 1) / kTileRows;
+        const int64_t xin = int64_t(m) * 128 * blocks_of(L[i].w.k);
+        for (int64_t t = 0; t < tiles; ++t) {
+            const int64_t rows = (t + 1 < tiles) ? kTileRows : L[i].w.n - t * kTileRows;
+            const int64_t tb = rows * rowb;
+            const int target = int((cum + tb / 2) * G / total);
+            cum += tb;
+            if (open && target != cur_target) close_range();
+            for (;;) {
+                if (!open) {
+                    if (nr == kMaxRanges) return fail(BITNET_ERR_INVALID_ARG, "stack needs more than %d CTAs", kMaxRanges);
+                    GemvRange &r = p.rng[nr];
+                    r.seg0 = int16_t(ns);
+                    r.nseg = 0;
+                    r.nin = 0;
+                    cur_x = 0;
+                    cur_target = target;
+                    open = true;
                 }
                 GemvRange &r = p.rng[nr];
                 int slot = -1;
                 for (int u = 0; u < r.nin; ++u)
                     if (r.in[u] == input_of[i]) slot = u;
+                const bool same_seg = r.nseg > 0 && p.seg[ns - 1].lin == i && p.seg[ns - 1].tile1 == t;
                 const bool need_in = slot < 0;
-                if (ns == kMaxSegs) {
-                    overflow = true;
-                    break;
-                }
-                if ((need_in && (r.nin == kMaxRangeInputs || cur_x + xin > xcap)) || r.nseg == kMaxRangeSegs) {
-                    close_range();   // r.nseg > 0 here: an empty range always fits one input
+                const bool need_seg = !same_seg;
+                if ((need_in && (r.nin == kMaxRangeInputs || cur_x + xin > xcap)) ||
+                    (need_seg && (r.nseg == kMaxRangeSegs || ns == kMaxSegs))) {
+                    if (r.nseg == 0 || ns == kMaxSegs)
+                        return fail(BITNET_ERR_INVALID_ARG, "stack too large for one launch (%d segments)", ns);
+                    close_range();
                     continue;
                 }
                 if (need_in) {
@@ -214,34 +394,42 @@ bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequa
                     r.in[r.nin++] = int16_t(input_of[i]);
                     cur_x += xin;
                 }
-                int64_t room = (target - cur_bytes + tb - 1) / tb;
-                if (room < 1) room = 1;
-                const int64_t take = (tiles - t) < room ? (tiles - t) : room;
-                GemvSeg &sg = p.seg[ns++];
-                sg.lin = int16_t(i);
-                sg.slot = int16_t(slot);
-                sg.tile0 = int32_t(t);
-                sg.tile1 = int32_t(t + take);
-                r.nseg++;
-                t += take;
-                cur_bytes += take * tb;
-                if (cur_bytes >= target) close_range();
+                if (need_seg) {
+                    GemvSeg &sg = p.seg[ns++];
+                    sg.lin = int16_t(i);
+                    sg.slot = int16_t(slot);
+                    sg.tile0 = int32_t(t);
+                    sg.tile1 = int32_t(t + 1);
+                    r.nseg++;
+                } else {
+                    p.seg[ns - 1].tile1 = int32_t(t + 1);
+                }
+                break;
             }
         }
-        if (overflow) continue;
-        close_range();
-        p.m = m;
-        p.num_ranges = nr;
-        p.prequant = prequant ? 1 : 0;
-        p.force_stall = g_force_stall;
-        p.flags = flags;
-        p.wait_limit = wait_limit();
-        p.x_bytes = int32_t((xmax + 127) / 128 * 128);
-        cudaError_t e = launch_gemv(p, nw, st);
-        if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
-        return BITNET_OK;
     }
-    return fail(BITNET_ERR_INVALID_ARG, "could not partition %d layers into %d ranges", count, kMaxRanges);
+    close_range();
+    p.m = m;
+    p.num_ranges = nr;
+    p.prequant = prequant ? 1 : 0;
+    p.force_stall = g_force_stall;
+    p.flags = flags;
+    p.wait_limit = wait_limit();
+    p.trace = g_trace;
+    p.x_bytes = int32_t((xmax + 127) / 128 * 128);
+    cudaError_t e = launch_gemv(p, variant, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
+    slot_plan.variant = variant;
+    slot_plan.key.layers = L;
+    slot_plan.key.m = m;
+    slot_plan.key.prequant = prequant;
+    slot_plan.key.flags = flags;
+    slot_plan.key.ordinal = dev.ordinal;
+    slot_plan.key.generation = gen;
+    slot_plan.key.wait_limit = g_wait_limit;
+    slot_plan.key.force_stall = g_force_stall;
+    slot_plan.key.trace = g_trace;
+    return BITNET_OK;
 }
 
 }  // namespace
@@ -290,6 +478,31 @@ int64_t bitnet_kpad(int64_t k)
 bitnet_status bitnet_debug_set_wait_limit(uint64_t cycles)
 {
     g_wait_limit = cycles;
+    return BITNET_OK;
+}
+
+bitnet_status bitnet_release_device_cache(void)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(BITNET_ERR_UNSUPPORTED_DEVICE, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_tmap_mu);
+    DeviceTmaps &D = g_tmaps[dev];
+    e = cudaDeviceSynchronize();
+    for (auto &c : D.chunks) {
+        cudaFree(c.dev);
+        cudaFreeHost(c.host);
+    }
+    D.chunks.clear();
+    D.index.clear();
+    ++g_tmap_generation;
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "cudaDeviceSynchronize");
+}
+
+bitnet_status bitnet_debug_set_trace(void *d_trace)
+{
+    g_trace = static_cast<uint64_t *>(d_trace);
     return BITNET_OK;
 }
 

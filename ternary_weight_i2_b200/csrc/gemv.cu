@@ -8,14 +8,17 @@
 // Decode is bound by reading the 2-bit weights once per token (technical
 // report §3.2, Figure 6b), so the kernel is built as a weight stream:
 //
-// * One CTA per SM works through a contiguous byte range of the launch's
-//   weights (host-balanced).  Each warp is an independent pipeline over the
-//   32-row tiles dealt to it: its lanes issue 1-D bulk (TMA) copies of their
-//   own row chunk into a padded shared-memory slot, two slots deep, and wait
-//   on an mbarrier; no register staging of weights.
+// * One CTA per SM works through a contiguous, byte-balanced range of the
+//   launch's weight tiles.  Each warp is an independent pipeline over the
+//   32-row tiles dealt to it: per unit it issues BOX 2-D tiled TMA loads
+//   (128 bytes x 32 rows each, 128-byte swizzle) from the layer's tensor map
+//   into a shared-memory slot, kSlotsPerWarp deep, and waits on an mbarrier;
+//   no register staging of weights.  Ragged tails (rows past N, bytes past
+//   the row end) are zero-filled by the tensor map and never used.
 // * Lane r owns weight row r of the tile, so there is no cross-lane reduction;
-//   the int8 activations are broadcast from shared memory (all lanes read the
-//   same address).
+//   the swizzle puts the 32 lanes' 16-byte reads of one column in distinct
+//   bank groups, and the int8 activations are broadcast from shared memory
+//   (all lanes read the same address).
 // * Decode in registers: a 32-bit word of codes holds 16 weights, four 2-bit
 //   fields per byte; masking field g (one LOP3) leaves 4^g * code in each byte,
 //   and dp4a multiplies those unsigned bytes by the signed activations.  With
@@ -23,9 +26,12 @@
 //   separate accumulators and are recombined as (64*a0+16*a1+4*a2+a3) >> 6.
 //   This is the unpack-then-multiply-add formulation of the technical report
 //   (codes as unsigned bytes times signed int8, like maddubs) on the dp4a unit.
+//   Even and odd blocks use separate accumulator sets for instruction-level
+//   parallelism.
 // * Every CTA quantises the activation rows its range needs straight into
 //   shared memory, laid out so one 16-byte read gives the four activation
-//   words a code word needs.
+//   words a code word needs.  The activation loads are issued before the
+//   weight prefetch so that they are not queued behind it.
 #include <cstdio>
 
 #include "common.cuh"
@@ -33,17 +39,32 @@
 
 namespace bitnet {
 
+struct SegInfo {
+    const void *tmap;
+    float *y;
+    int32_t *acc;
+    int32_t n;
+    int32_t rowb;    // packed bytes per row
+    int32_t kb;      // blocks per row
+    int32_t nch;     // chunks per tile
+    int32_t slot;    // range-local input slot
+    int32_t tile0;   // first tile of the layer in this range
+    int32_t tcum;    // range-local index of the segment's first tile
+    float scale;
+};
+
 template <int M>
 struct GemvMeta {
-    uint64_t bar[8 * kSlotsPerWarp];
+    uint64_t bar[kMaxWarps * kSlotsPerWarp];
     uint64_t stall_bar;
-    int32_t tcum[kMaxRangeSegs + 1];
-    int32_t seg_lin[kMaxRangeSegs];
-    int32_t seg_slot[kMaxRangeSegs];
-    int32_t seg_tile0[kMaxRangeSegs];
+    SegInfo seg[kMaxRangeSegs];
+    int32_t ttot;
     int32_t xoff[kMaxRangeInputs];
     int32_t kpad[kMaxRangeInputs];
     int32_t wstart[kMaxRangeInputs * M + 1];   // job word starts (job = slot*M + m)
+    const void *xptr[kMaxRangeInputs];
+    const float *xscale[kMaxRangeInputs];
+    int32_t xk[kMaxRangeInputs];
     uint32_t amax[kMaxRangeInputs * M];
     int32_t nonfin[kMaxRangeInputs * M];
     float inv[kMaxRangeInputs * M];
@@ -59,13 +80,45 @@ __device__ __forceinline__ uint32_t perm_offset(int p)
     return uint32_t((p >> 5) * 128 + (p & 7) * 16 + ((p >> 3) & 3) * 4);
 }
 
-template <int M, int NW>
+// Block jj of a unit for lane r: box jj/4, 128-byte line r of that box, 16-byte
+// chunks 2*(jj%4)+h placed by the 128-byte swizzle (chunk ^ (r & 7)).
+template <int M>
+__device__ __forceinline__ void block_dot(uint32_t wrow, uint32_t rx, uint32_t xb, int kp, int jj,
+                                          int32_t (&acc)[M][4])
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t ch = uint32_t((jj & 3) * 2 + h) ^ rx;
+        const uint4 wv = lds128(wrow + (jj >> 2) * kBoxBytes + ch * 16);
+        const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t c0 = wd[i] & 0x03030303u, c1 = wd[i] & 0x0C0C0C0Cu;
+            const uint32_t c2 = wd[i] & 0x30303030u, c3 = wd[i] & 0xC0C0C0C0u;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const uint4 xv = lds128(xb + m * kp + jj * 128 + (4 * h + i) * 16);
+                acc[m][0] = dp4a_us(c0, xv.x, acc[m][0]);
+                acc[m][1] = dp4a_us(c1, xv.y, acc[m][1]);
+                acc[m][2] = dp4a_us(c2, xv.z, acc[m][2]);
+                acc[m][3] = dp4a_us(c3, xv.w, acc[m][3]);
+            }
+        }
+    }
+}
+
+template <int M, int NW, int BOX>
 __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_constant__ GemvParams p)
 {
     constexpr int T = NW * 32;
-    constexpr int QB = 16;   // float4 words a thread holds per quantiser batch
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *xarea = smem + gemv_ring_bytes(NW);
+    constexpr int QB = (NW >= 16) ? 8 : 16;   // float4 words a thread holds per quantiser batch
+    constexpr int SLOT = slot_bytes(BOX);
+    constexpr int UNIT_BYTES = BOX * 128;     // bytes of each row per unit
+    constexpr int UNIT_BLOCKS = BOX * kBoxBlocks;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // swizzled boxes need 1024-byte aligned destinations
+    uint8_t *smem = smem_raw + ((kAlignPad - (smem_u32(smem_raw) & (kAlignPad - 1))) & (kAlignPad - 1));
+    uint8_t *xarea = smem + ring_bytes(NW, BOX);
     GemvMeta<M> *meta = reinterpret_cast<GemvMeta<M> *>(xarea + p.x_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -74,28 +127,57 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
     const uint64_t limit = p.wait_limit;
 
     // ---------------------------------------------------------- set-up
-    if (tid == 0) {
-        meta->tcum[0] = 0;
-        for (int s = 0; s < nseg; ++s) {
-            const GemvSeg &sg = p.seg[R.seg0 + s];
-            meta->tcum[s + 1] = meta->tcum[s] + (sg.tile1 - sg.tile0);
-            meta->seg_lin[s] = sg.lin;
-            meta->seg_slot[s] = sg.slot;
-            meta->seg_tile0[s] = sg.tile0;
+    // warp 0: one lane per segment; warp 1: one lane per input slot
+    if (warp == 0) {
+        int cnt = 0;
+        if (lane < nseg) {
+            const GemvSeg sg = p.seg[R.seg0 + lane];
+            const GemvLinear &L = p.lin[sg.lin];
+            SegInfo &si = meta->seg[lane];
+            si.tmap = L.tmap;
+            si.y = L.y;
+            si.acc = L.acc;
+            si.n = L.n;
+            si.kb = L.kb;
+            si.rowb = 32 * L.kb;
+            si.nch = (32 * L.kb + UNIT_BYTES - 1) / UNIT_BYTES;
+            si.slot = sg.slot;
+            si.tile0 = sg.tile0;
+            si.scale = L.scale;
+            cnt = sg.tile1 - sg.tile0;
         }
-        int off = 0, w = 0;
-        for (int u = 0; u < nin; ++u) {
-            const int kp = 128 * p.inp[R.in[u]].kb;
-            meta->xoff[u] = off;
-            meta->kpad[u] = kp;
-            off += M * kp;
-            for (int m = 0; m < M; ++m) {
-                meta->wstart[u * M + m] = w;
-                w += kp / 4;
-            }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        meta->wstart[nin * M] = w;
-        mbar_init(smem_u32(&meta->stall_bar), 1);
+        if (lane < nseg) meta->seg[lane].tcum = incl - cnt;
+        if (lane == 31) meta->ttot = incl;
+        if (lane == 0) mbar_init(smem_u32(&meta->stall_bar), 1);
+    } else if (warp == 1) {
+        int bytes = 0, kp = 0;
+        if (lane < nin) {
+            const GemvInput &in = p.inp[R.in[lane]];
+            kp = 128 * in.kb;
+            bytes = M * kp;
+            meta->xptr[lane] = in.x;
+            meta->xscale[lane] = in.scale;
+            meta->xk[lane] = in.k;
+            meta->kpad[lane] = kp;
+        }
+        int incl = bytes;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane < nin) {
+            const int off = incl - bytes;
+            meta->xoff[lane] = off;
+            for (int m = 0; m < M; ++m) meta->wstart[lane * M + m] = (off + m * kp) / 4;
+        }
+        if (lane == 31) meta->wstart[nin * M] = incl / 4;
     }
     if (lane == 0)
         for (int s = 0; s < kSlotsPerWarp; ++s) mbar_init(smem_u32(&meta->bar[warp * kSlotsPerWarp + s]), 1);
@@ -106,6 +188,11 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
     }
     fence_mbar_init();
     __syncthreads();
+    uint64_t *trace = p.trace ? p.trace + (size_t(blockIdx.x) * NW + warp) * kTraceEvents : nullptr;
+    auto stamp = [&](int ev) {
+        if (trace && lane == 0) trace[ev] = globaltimer();
+    };
+    stamp(0);
 
     if (p.force_stall) {
         // Test aid: wait on a barrier nobody arrives at; the bounded wait
@@ -114,167 +201,165 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
         return;
     }
 
-    const int ttot = meta->tcum[nseg];
-    const uint32_t ring = smem_u32(smem) + warp * kSlotsPerWarp * kSlotBytes;
-    const uint32_t bar0 = smem_u32(&meta->bar[warp * kSlotsPerWarp]);
+    // ------------------------------- activation loads (pass-1 registers)
+    const int W = meta->wstart[nin * M];
+    const int nbatch = (W + QB * T - 1) / (QB * T);
+    float4 xr[QB];
+    auto load_word = [&](int J, int word) -> float4 {
+        const int u = J / M, m = J - u * M;
+        const int k = meta->xk[u];
+        const int pw = word - meta->wstart[J];
+        const int k0 = 4 * pw;
+        const float *row = static_cast<const float *>(meta->xptr[u]) + size_t(m) * size_t(k);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k0 + 3 < k && (reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+            v = __ldg(reinterpret_cast<const float4 *>(row + k0));
+        } else {
+            if (k0 + 0 < k) v.x = __ldg(row + k0 + 0);
+            if (k0 + 1 < k) v.y = __ldg(row + k0 + 1);
+            if (k0 + 2 < k) v.z = __ldg(row + k0 + 2);
+            if (k0 + 3 < k) v.w = __ldg(row + k0 + 3);
+        }
+        return v;
+    };
+    auto load_batch = [&](int b) {
+        int J = 0;
+#pragma unroll
+        for (int q = 0; q < QB; ++q) {
+            const int word = (b * QB + q) * T + tid;   // warp-uniform job
+            if (word - lane >= W) break;
+            while (word - lane >= meta->wstart[J + 1]) ++J;
+            xr[q] = load_word(J, word);
+        }
+    };
+    if (!p.prequant) load_batch(0);
 
-    auto nchunks = [&](int s) { return (p.lin[meta->seg_lin[s]].kb + kChunkBlocks - 1) / kChunkBlocks; };
+    // ------------------------------------------------ weight prefetch
+    const int ttot = meta->ttot;
+    const uint64_t policy = l2_evict_first_policy();
+    const uint32_t ring = smem_u32(smem) + warp * kSlotsPerWarp * SLOT;
+    const uint32_t bar0 = smem_u32(&meta->bar[warp * kSlotsPerWarp]);
+    auto seg_end = [&](int s) { return s + 1 < nseg ? meta->seg[s + 1].tcum : ttot; };
     auto advance = [&](int &i, int &s, int &c) {
-        if (++c == nchunks(s)) {
+        if (++c == meta->seg[s].nch) {
             c = 0;
             i += NW;
-            while (s < nseg && i >= meta->tcum[s + 1]) ++s;
+            while (s < nseg && i >= seg_end(s)) ++s;
         }
     };
     auto issue = [&](int i, int s, int c, int slot) {
-        const GemvLinear &L = p.lin[meta->seg_lin[s]];
-        const int row0 = (meta->seg_tile0[s] + (i - meta->tcum[s])) * kTileRows;
-        const int rows = min(kTileRows, L.n - row0);
-        const int cb0 = c * kChunkBlocks;
-        const int bytes = 32 * min(kChunkBlocks, L.kb - cb0);
+        const SegInfo &si = meta->seg[s];
+        const int row0 = (si.tile0 + (i - si.tcum)) * kTileRows;
+        const int x0 = c * UNIT_BYTES;
+        const int nbox = min(BOX, (si.rowb - x0 + 127) / 128);   // boxes that start inside the row
         const uint32_t bar = bar0 + 8 * slot;
-        if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(rows * bytes));
+        if (lane == 0) mbar_arrive_expect_tx(bar, uint32_t(nbox * kBoxBytes));
         __syncwarp();
-        if (lane < rows)
-            bulk_g2s(ring + slot * kSlotBytes + lane * kSlotPitch,
-                     L.packed + size_t(row0 + lane) * size_t(32 * L.kb) + 32 * cb0, uint32_t(bytes), bar);
+        if (lane < nbox)
+            tma_load_2d(ring + slot * SLOT + lane * kBoxBytes, si.tmap, x0 + lane * 128, row0, bar, policy);
     };
-
-    // producer iterator: start streaming weights before quantising
     int pi = warp, ps = 0, pc = 0;
-    while (ps < nseg && pi >= meta->tcum[ps + 1]) ++ps;
+    while (ps < nseg && pi >= seg_end(ps)) ++ps;
     int issued = 0;
     for (int sl = 0; sl < kSlotsPerWarp && pi < ttot; ++sl) {
         issue(pi, ps, pc, sl);
         advance(pi, ps, pc);
         ++issued;
     }
+    stamp(1);
 
     // ------------------------------------------- activation quantiser
-    {
-        const int W = meta->wstart[nin * M];
-        const int nbatch = (W + QB * T - 1) / (QB * T);
-        float4 xr[QB];
-        auto load_word = [&](int J, int word) -> float4 {
-            const int u = J / M, m = J - u * M;
-            const GemvInput &in = p.inp[R.in[u]];
-            const int pw = word - meta->wstart[J];
-            const int k0 = 4 * pw;
-            const float *row = static_cast<const float *>(in.x) + size_t(m) * size_t(in.k);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k0 + 3 < in.k && (reinterpret_cast<uintptr_t>(row) & 15) == 0) {
-                v = __ldg(reinterpret_cast<const float4 *>(row + k0));
-            } else {
-                if (k0 + 0 < in.k) v.x = __ldg(row + k0 + 0);
-                if (k0 + 1 < in.k) v.y = __ldg(row + k0 + 1);
-                if (k0 + 2 < in.k) v.z = __ldg(row + k0 + 2);
-                if (k0 + 3 < in.k) v.w = __ldg(row + k0 + 3);
-            }
-            return v;
-        };
-        if (!p.prequant) {
-            // pass 1: absmax and finiteness per job (token row of an input)
-            for (int b = 0; b < nbatch; ++b) {
-                int J = 0;
+    if (!p.prequant) {
+        // pass 1: absmax and finiteness per job (token row of an input)
+        for (int b = 0; b < nbatch; ++b) {
+            if (b > 0) load_batch(b);
+            int J = 0;
 #pragma unroll
-                for (int q = 0; q < QB; ++q) {
-                    const int word = (b * QB + q) * T + tid;   // warp-uniform job
-                    if (word - lane >= W) break;
-                    while (word - lane >= meta->wstart[J + 1]) ++J;
-                    xr[q] = word < W ? load_word(J, word) : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                J = 0;
-#pragma unroll
-                for (int q = 0; q < QB; ++q) {
-                    const int word = (b * QB + q) * T + tid;
-                    if (word - lane >= W) break;
-                    while (word - lane >= meta->wstart[J + 1]) ++J;
-                    const float4 v = xr[q];
-                    const bool fin = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-                    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-                    if (!fin) a = 0.f;
-                    a = warp_max(a);
-                    const bool anynf = __any_sync(0xffffffffu, !fin);
-                    if (lane == 0) {
-                        atomicMax(&meta->amax[J], __float_as_uint(a));
-                        if (anynf) meta->nonfin[J] = 1;
-                    }
-                }
-            }
-            __syncthreads();
-            for (int J = tid; J < nin * M; J += T) {
-                const float amax = __uint_as_float(meta->amax[J]);
-                const bool bad = meta->nonfin[J] != 0;
-                if (bad) raise_flag(p.flags, BITNET_FLAG_NONFINITE);
-                meta->inv[J] = (bad || amax == 0.f) ? 0.f : __fdiv_rn(127.0f, amax);
-                meta->s_act[J] = (bad || amax == 0.f) ? 0.f : __fdiv_rn(amax, 127.0f);
-            }
-            __syncthreads();
-            // pass 2: codes into the broadcast layout, and sum(q) per job
-            for (int b = 0; b < nbatch; ++b) {
-                int J = 0;
-#pragma unroll
-                for (int q = 0; q < QB; ++q) {
-                    const int word = (b * QB + q) * T + tid;
-                    if (word - lane >= W) break;
-                    while (word - lane >= meta->wstart[J + 1]) ++J;
-                    const float4 v = (nbatch == 1) ? xr[q]
-                                                   : (word < W ? load_word(J, word) : make_float4(0.f, 0.f, 0.f, 0.f));
-                    const float inv = meta->inv[J];
-                    int32_t q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-                    if (word < W && inv != 0.f) {
-                        q0 = quant_one(v.x, inv);
-                        q1 = quant_one(v.y, inv);
-                        q2 = quant_one(v.z, inv);
-                        q3 = quant_one(v.w, inv);
-                    }
-                    const int32_t s = warp_sum(q0 + q1 + q2 + q3);
-                    if (word < W) {
-                        const int u = J / M, m = J - u * M;
-                        const int pw = word - meta->wstart[J];
-                        *reinterpret_cast<uint32_t *>(xarea + meta->xoff[u] + m * meta->kpad[u] + perm_offset(pw)) =
-                            pack4(q0, q1, q2, q3);
-                    }
-                    if (lane == 0) atomicAdd(&meta->sumx[J], s);
-                }
-            }
-        } else {
-            // pre-quantised int8 rows [m, kpad] with given scales
-            for (int word = tid; word - lane < W; word += T) {
-                int J = 0;
+            for (int q = 0; q < QB; ++q) {
+                const int word = (b * QB + q) * T + tid;
+                if (word - lane >= W) break;
                 while (word - lane >= meta->wstart[J + 1]) ++J;
-                const int u = J / M, m = J - u * M;
-                const GemvInput &in = p.inp[R.in[u]];
-                const int pw = word - meta->wstart[J];
-                uint32_t v = 0;
-                int32_t s = 0;
-                if (word < W) {
-                    v = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const int8_t *>(in.x) +
-                                                                 size_t(m) * size_t(meta->kpad[u])) +
-                              pw);
-                    s = int32_t(int8_t(v)) + int32_t(int8_t(v >> 8)) + int32_t(int8_t(v >> 16)) +
-                        int32_t(int8_t(v >> 24));
-                    *reinterpret_cast<uint32_t *>(xarea + meta->xoff[u] + m * meta->kpad[u] + perm_offset(pw)) = v;
+                const float4 v = xr[q];
+                const bool fin = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+                float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+                if (!fin) a = 0.f;
+                a = warp_max(a);
+                const bool anynf = __any_sync(0xffffffffu, !fin);
+                if (lane == 0) {
+                    atomicMax(&meta->amax[J], __float_as_uint(a));
+                    if (anynf) meta->nonfin[J] = 1;
                 }
-                s = warp_sum(s);
+            }
+        }
+        __syncthreads();
+        for (int J = tid; J < nin * M; J += T) {
+            const float amax = __uint_as_float(meta->amax[J]);
+            const bool bad = meta->nonfin[J] != 0;
+            if (bad) raise_flag(p.flags, BITNET_FLAG_NONFINITE);
+            meta->inv[J] = (bad || amax == 0.f) ? 0.f : __fdiv_rn(127.0f, amax);
+            meta->s_act[J] = (bad || amax == 0.f) ? 0.f : __fdiv_rn(amax, 127.0f);
+        }
+        __syncthreads();
+        // pass 2: codes into the broadcast layout, and sum(q) per job
+        for (int b = 0; b < nbatch; ++b) {
+            if (nbatch > 1) load_batch(b);
+            int J = 0;
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+                const int word = (b * QB + q) * T + tid;
+                if (word - lane >= W) break;
+                while (word - lane >= meta->wstart[J + 1]) ++J;
+                const float4 v = xr[q];
+                const float inv = meta->inv[J];
+                int32_t q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+                if (inv != 0.f) {
+                    q0 = quant_one(v.x, inv);
+                    q1 = quant_one(v.y, inv);
+                    q2 = quant_one(v.z, inv);
+                    q3 = quant_one(v.w, inv);
+                }
+                const int32_t s = warp_sum(q0 + q1 + q2 + q3);
+                const int u = J / M, m = J - u * M;
+                const int pw = word - meta->wstart[J];
+                *reinterpret_cast<uint32_t *>(xarea + meta->xoff[u] + m * meta->kpad[u] + perm_offset(pw)) =
+                    pack4(q0, q1, q2, q3);
                 if (lane == 0) atomicAdd(&meta->sumx[J], s);
             }
-            for (int J = tid; J < nin * M; J += T) {
-                const int u = J / M, m = J - u * M;
-                meta->s_act[J] = p.inp[R.in[u]].scale[m];
-            }
+        }
+    } else {
+        // pre-quantised int8 rows [m, kpad] with given scales
+        for (int word = tid; word - lane < W; word += T) {
+            int J = 0;
+            while (word - lane >= meta->wstart[J + 1]) ++J;
+            const int u = J / M, m = J - u * M;
+            const int pw = word - meta->wstart[J];
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(static_cast<const int8_t *>(meta->xptr[u]) +
+                                                                       size_t(m) * size_t(meta->kpad[u])) +
+                                     pw);
+            int32_t s = int32_t(int8_t(v)) + int32_t(int8_t(v >> 8)) + int32_t(int8_t(v >> 16)) +
+                        int32_t(int8_t(v >> 24));
+            *reinterpret_cast<uint32_t *>(xarea + meta->xoff[u] + m * meta->kpad[u] + perm_offset(pw)) = v;
+            s = warp_sum(s);
+            if (lane == 0) atomicAdd(&meta->sumx[J], s);
+        }
+        for (int J = tid; J < nin * M; J += T) {
+            const int u = J / M, m = J - u * M;
+            meta->s_act[J] = meta->xscale[u][m];
         }
     }
     __syncthreads();
+    stamp(2);
 
     // ------------------------------------------------- stream and multiply
     int ci = warp, cs = 0, cc = 0;
-    while (cs < nseg && ci >= meta->tcum[cs + 1]) ++cs;
+    while (cs < nseg && ci >= seg_end(cs)) ++cs;
     int slot = 0, consumed = 0;
     uint32_t phase = 0;
-    int32_t acc[M][4];
+    int32_t acc0[M][4], acc1[M][4];
 #pragma unroll
-    for (int m = 0; m < M; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0;
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) acc0[m][g] = acc1[m][g] = 0;
     bool timed_out = false;
 
     while (ci < ttot) {
@@ -284,50 +369,39 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
             break;
         }
         phase ^= 1u << slot;
-        const int lin = meta->seg_lin[cs];
-        const GemvLinear &L = p.lin[lin];
-        const int u = meta->seg_slot[cs];
+        if (consumed == 0) stamp(3);
+        const SegInfo &si = meta->seg[cs];
+        const int u = si.slot;
         const int kp = meta->kpad[u];
-        const int cb0 = cc * kChunkBlocks;
-        const int nblk = min(kChunkBlocks, L.kb - cb0);
-        const uint32_t wrow = ring + slot * kSlotBytes + lane * kSlotPitch;
+        const int cb0 = cc * UNIT_BLOCKS;
+        const int nblk = min(UNIT_BLOCKS, si.kb - cb0);
+        const uint32_t wrow = ring + slot * SLOT + lane * 128;
+        const uint32_t rx = uint32_t(lane & 7);
         const uint32_t xb = smem_u32(xarea) + meta->xoff[u] + cb0 * 128;
-#pragma unroll 2
-        for (int jj = 0; jj < nblk; ++jj) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 wv = lds128(wrow + jj * 32 + h * 16);
-                const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t c0 = wd[i] & 0x03030303u, c1 = wd[i] & 0x0C0C0C0Cu;
-                    const uint32_t c2 = wd[i] & 0x30303030u, c3 = wd[i] & 0xC0C0C0C0u;
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        const uint4 xv = lds128(xb + m * kp + jj * 128 + (4 * h + i) * 16);
-                        acc[m][0] = dp4a_us(c0, xv.x, acc[m][0]);
-                        acc[m][1] = dp4a_us(c1, xv.y, acc[m][1]);
-                        acc[m][2] = dp4a_us(c2, xv.z, acc[m][2]);
-                        acc[m][3] = dp4a_us(c3, xv.w, acc[m][3]);
-                    }
-                }
-            }
+        int jj = 0;
+#pragma unroll 1
+        for (; jj + 1 < nblk; jj += 2) {
+            block_dot<M>(wrow, rx, xb, kp, jj, acc0);
+            block_dot<M>(wrow, rx, xb, kp, jj + 1, acc1);
         }
-        if (cc == nchunks(cs) - 1) {
-            const int row0 = (meta->seg_tile0[cs] + (ci - meta->tcum[cs])) * kTileRows;
-            const int row = row0 + lane;
-            if (row < L.n) {
+        if (jj < nblk) block_dot<M>(wrow, rx, xb, kp, jj, acc0);
+        if (cc == si.nch - 1) {
+            const int row = (si.tile0 + (ci - si.tcum)) * kTileRows + lane;
+            if (row < si.n) {
 #pragma unroll
                 for (int m = 0; m < M; ++m) {
-                    const int32_t s64 = acc[m][0] * 64 + acc[m][1] * 16 + acc[m][2] * 4 + acc[m][3];
+                    const int32_t s64 = (acc0[m][0] + acc1[m][0]) * 64 + (acc0[m][1] + acc1[m][1]) * 16 +
+                                        (acc0[m][2] + acc1[m][2]) * 4 + (acc0[m][3] + acc1[m][3]);
                     const int32_t a = (s64 >> 6) - meta->sumx[u * M + m];
-                    const float yv = __fmul_rn(__fmul_rn(float(a), meta->s_act[u * M + m]), L.scale);
-                    L.y[size_t(m) * size_t(L.n) + row] = yv;
-                    if (L.acc) L.acc[size_t(m) * size_t(L.n) + row] = a;
+                    const float yv = __fmul_rn(__fmul_rn(float(a), meta->s_act[u * M + m]), si.scale);
+                    si.y[size_t(m) * size_t(si.n) + row] = yv;
+                    if (si.acc) si.acc[size_t(m) * size_t(si.n) + row] = a;
                 }
             }
 #pragma unroll
-            for (int m = 0; m < M; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0;
+            for (int m = 0; m < M; ++m)
+#pragma unroll
+                for (int g = 0; g < 4; ++g) acc0[m][g] = acc1[m][g] = 0;
         }
         __syncwarp();
         ++consumed;
@@ -339,6 +413,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
         advance(ci, cs, cc);
         slot = (slot + 1 == kSlotsPerWarp) ? 0 : slot + 1;
     }
+    stamp(4);
 
     if (timed_out) {
         raise_flag(p.flags, BITNET_FLAG_TIMEOUT);
@@ -353,44 +428,49 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
 
 // ------------------------------------------------------------- launcher
 
-template <int M, int NW>
+template <int M, int NW, int BOX>
 static cudaError_t launch_one(const GemvParams &p, size_t smem, cudaStream_t st)
 {
     static bool configured = false;   // per instantiation, set once
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_stack_kernel<M, NW>,
+        cudaError_t e = cudaFuncSetAttribute(gemv_stack_kernel<M, NW, BOX>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    gemv_stack_kernel<M, NW><<<p.num_ranges, NW * 32, smem, st>>>(p);
+    gemv_stack_kernel<M, NW, BOX><<<p.num_ranges, NW * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 
-template <int NW>
-static cudaError_t launch_nw(const GemvParams &p, size_t smem, cudaStream_t st)
+template <int NW, int BOX, int MAXM>
+static cudaError_t launch_variant(const GemvParams &p, size_t smem, cudaStream_t st)
 {
     switch (p.m) {
-    case 1: return launch_one<1, NW>(p, smem, st);
-    case 2: return launch_one<2, NW>(p, smem, st);
-    case 3: return launch_one<3, NW>(p, smem, st);
-    case 4: return launch_one<4, NW>(p, smem, st);
-    case 5: return launch_one<5, NW>(p, smem, st);
-    case 6: return launch_one<6, NW>(p, smem, st);
-    case 7: return launch_one<7, NW>(p, smem, st);
-    case 8: return launch_one<8, NW>(p, smem, st);
-    default: return cudaErrorInvalidValue;
+    case 1: return launch_one<1, NW, BOX>(p, smem, st);
+    case 2: if constexpr (MAXM >= 2) return launch_one<2, NW, BOX>(p, smem, st); break;
+    case 3: if constexpr (MAXM >= 3) return launch_one<3, NW, BOX>(p, smem, st); break;
+    case 4: if constexpr (MAXM >= 4) return launch_one<4, NW, BOX>(p, smem, st); break;
+    case 5: if constexpr (MAXM >= 5) return launch_one<5, NW, BOX>(p, smem, st); break;
+    case 6: if constexpr (MAXM >= 6) return launch_one<6, NW, BOX>(p, smem, st); break;
+    case 7: if constexpr (MAXM >= 7) return launch_one<7, NW, BOX>(p, smem, st); break;
+    case 8: if constexpr (MAXM >= 8) return launch_one<8, NW, BOX>(p, smem, st); break;
+    default: break;
     }
+    return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemv(const GemvParams &p, int nw, cudaStream_t st)
+cudaError_t launch_gemv(const GemvParams &p, int variant, cudaStream_t st)
 {
-    const size_t smem = size_t(gemv_ring_bytes(nw)) + size_t(p.x_bytes) + size_t(kMetaBytes);
+    if (variant < 0 || variant >= kNumVariants || p.m > kVariantMaxM[variant]) return cudaErrorInvalidValue;
+    const GemvVariant v = kVariants[variant];
+    const size_t smem =
+        size_t(kAlignPad) + size_t(ring_bytes(v.nw, v.boxes)) + size_t(p.x_bytes) + size_t(kMetaBytes);
     if (smem > size_t(kSmemLimit)) return cudaErrorInvalidValue;
-    switch (nw) {
-    case 8: return launch_nw<8>(p, smem, st);
-    case 6: return launch_nw<6>(p, smem, st);
-    case 4: return launch_nw<4>(p, smem, st);
+    switch (variant) {
+    case 0: return launch_variant<kVariants[0].nw, kVariants[0].boxes, kVariantMaxM[0]>(p, smem, st);
+    case 1: return launch_variant<kVariants[1].nw, kVariants[1].boxes, kVariantMaxM[1]>(p, smem, st);
+    case 2: return launch_variant<kVariants[2].nw, kVariants[2].boxes, kVariantMaxM[2]>(p, smem, st);
+    case 3: return launch_variant<kVariants[3].nw, kVariants[3].boxes, kVariantMaxM[3]>(p, smem, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -153,11 +153,14 @@ def test_edge_sweep(m, k, n):
 def test_saturation_max_k(m):
     k, n = 9024, 64
     x = np.full((m, k), 0.5, np.float32)
-    x[m - 1] = -0.5
+    if m > 1:
+        x[m - 1] = -0.5
     w = np.ones((n, k), np.int8)
     w[1::2] = -1
     ag, _ = _check_linear(x, w, 0.05)
-    assert ag[0, 0] == 127 * 9024
+    assert ag[0, 0] == 127 * 9024 and ag[0, 1] == -127 * 9024
+    if m > 1:
+        assert ag[m - 1, 0] == -127 * 9024
 
 
 @pytest.mark.parametrize("m", [1, 4, 8])
