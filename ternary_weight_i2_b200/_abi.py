@@ -204,3 +204,4 @@ class StackCall:
 
 def linear_stack(xs, tws, ys, accs=None, flags=None, stream=None) -> None:
     StackCall(xs, tws, ys, accs)(flags=flags, stream=stream)
+

@@ -417,6 +417,9 @@ bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequa
     p.wait_limit = wait_limit();
     p.trace = g_trace;
     p.x_bytes = int32_t((xmax + 127) / 128 * 128);
+    // cache entries are never rewritten, but after a release a new chunk can
+    // reuse the address of a freed one
+    p.fence_maps = gen > 1 ? 1 : 0;
     cudaError_t e = launch_gemv(p, variant, st);
     if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
     slot_plan.variant = variant;
@@ -674,3 +677,4 @@ bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet
 }
 
 }  // extern "C"
+

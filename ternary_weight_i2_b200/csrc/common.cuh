@@ -99,6 +99,14 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// Order this thread's later TMA uses of the tensor map at `tmap` (global
+// memory) after writes to it made before the launch (host copies): a map's
+// bytes may have been rewritten at an address the TMA unit has seen before.
+__device__ __forceinline__ void tensormap_acquire(const void *tmap)
+{
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(tmap) : "memory");
+}
+
 // L2 policy for data read exactly once per launch (the weight stream): evict
 // first, so that it does not push activations and outputs out of L2.
 __device__ __forceinline__ uint64_t l2_evict_first_policy()

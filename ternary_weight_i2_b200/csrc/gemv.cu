@@ -258,6 +258,10 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
         if (lane < nbox)
             tma_load_2d(ring + slot * SLOT + lane * kBoxBytes, si.tmap, x0 + lane * 128, row0, bar, policy);
     };
+    // lanes that issue TMA loads acquire every map of the range once when the
+    // maps' bytes may have changed at an address the TMA unit has cached
+    if (p.fence_maps && lane < BOX)
+        for (int s = 0; s < nseg; ++s) tensormap_acquire(meta->seg[s].tmap);
     int pi = warp, ps = 0, pc = 0;
     while (ps < nseg && pi >= seg_end(ps)) ++ps;
     int issued = 0;

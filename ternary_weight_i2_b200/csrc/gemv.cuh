@@ -77,7 +77,7 @@ struct GemvParams {
     int32_t *flags;
     uint64_t wait_limit;
     int32_t x_bytes;         // bytes of the shared-memory activation area
-    int32_t pad_;
+    int32_t fence_maps;      // tensor maps may have been rewritten at a reused address
     uint64_t *trace;         // optional: kTraceEvents globaltimer stamps per warp
     GemvLinear lin[kMaxLinears];
     GemvInput inp[kMaxInputs];
