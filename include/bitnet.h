@@ -204,6 +204,33 @@ BITNET_API bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, c
                                   int64_t count, float *const *y, int32_t *const *acc_out,
                                   int32_t *d_flags, void *stream);
 
+/*
+ * bitnet_linear_stack with no device allocation, for callers that cannot call
+ * cudaMalloc: code running where the allocator is owned by someone else (a
+ * host framework with its own pooling allocator, a real-time loop that must not
+ * take the allocator's locks, a process whose memory is reserved up front) or
+ * that must not grow the device footprint after start-up.  The technical report
+ * has no counterpart to this entry point.
+ *
+ * Same arguments, layouts, results and errors as bitnet_linear_stack.  The
+ * per-layer TMA tensor maps, which bitnet_linear_stack keeps in an allocated
+ * per-device cache, are written instead into one fixed array of 256 maps
+ * (32 KB) that is part of the library's device image: every GPU that loads the
+ * library holds it until the process exits.  Limit: count <= 256
+ * (BITNET_STACK_MAX); a larger count returns BITNET_ERR_INVALID_ARG.
+ * - No cudaMalloc, cudaFree, pinned or other allocation is made.
+ * - The first call on a device looks up the array's device address; make that
+ *   first call before any stream capture.
+ * - The array is shared by every call and keeps the last call's maps.  A call
+ *   whose weight descriptors differ from the ones the array holds rewrites it
+ *   with a copy from host memory on `stream` (that copy waits for earlier work
+ *   on `stream`).  Calls that overlap on the GPU (other streams, other host
+ *   threads) race on the array and must not be made.
+ */
+BITNET_API bitnet_status bitnet_linear_stack_noalloc(const float *const *x, int64_t m, const bitnet_tw *w,
+                                                     int64_t count, float *const *y, int32_t *const *acc_out,
+                                                     int32_t *d_flags, void *stream);
+
 /* Free the current device's tensor-map cache (waits for the device to be
  * idle first).  Later calls rebuild entries as needed. */
 BITNET_API bitnet_status bitnet_release_device_cache(void);

@@ -49,6 +49,7 @@ _SIGNATURES = {
     "bitnet_linear": ([_P, _I64, C.POINTER(TW), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
     "bitnet_linear_q": ([_P, _P, _I64, C.POINTER(TW), _P, _P, _P, _P], C.c_int),
     "bitnet_linear_stack": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
+    "bitnet_linear_stack_noalloc": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
     "bitnet_debug_set_trace": ([_P], C.c_int),
@@ -205,3 +206,10 @@ class StackCall:
 def linear_stack(xs, tws, ys, accs=None, flags=None, stream=None) -> None:
     StackCall(xs, tws, ys, accs)(flags=flags, stream=stream)
 
+
+def linear_stack_noalloc(xs, tws, ys, accs=None, flags=None, stream=None) -> None:
+    """bitnet_linear_stack_noalloc: the stack call that allocates no device
+    memory (tensor maps in the library's fixed device array)."""
+    c = StackCall(xs, tws, ys, accs)
+    _check(load().bitnet_linear_stack_noalloc(c.x_arr, c.m, c.tw_arr, c.count, c.y_arr, c.acc_arr,
+                                              _ptr(flags), _stream(stream)), "bitnet_linear_stack_noalloc")

@@ -678,3 +678,236 @@ bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet
 
 }  // extern "C"
 
+// ===================================================================
+// bitnet_linear_stack_noalloc: the decode stack for callers that cannot
+// allocate device memory.
+//
+// The ordinary stack call keeps each weight tensor's TMA tensor map in a
+// per-device cache that it allocates with cudaMalloc/cudaMallocHost the first
+// time it meets the tensor.  This variant instead writes the maps into the
+// fixed array below, which is part of the library's module image (every GPU
+// that loads the library holds it until the process exits), and otherwise runs
+// the same kernel.  Its limit is the array's size: kNoallocMaxLayers maps.
+// ===================================================================
+
+static constexpr int kNoallocMaxLayers = BITNET_STACK_MAX;   // 256 maps x 128 bytes = 32 KB
+static __device__ __align__(256) uint8_t g_noalloc_tmaps[kNoallocMaxLayers * sizeof(CUtensorMap)];
+
+namespace {
+
+std::mutex g_na_mu;                        // guards everything below
+void *g_na_dev_addr[64] = {nullptr};       // device address of g_noalloc_tmaps, per device
+struct NaKey {
+    const void *p;
+    int64_t n, k;
+};
+NaKey g_na_copied[64][kNoallocMaxLayers];  // descriptors whose maps each device's array holds
+int g_na_copied_count[64] = {0};
+CUtensorMap g_na_host_maps[kNoallocMaxLayers];
+LayerReq g_na_layers[kNoallocMaxLayers];
+int g_na_input_of[kNoallocMaxLayers];
+GemvParams g_na_params;
+
+// Set-up, once per device, with that device current: the array's name is only
+// a host-side stand-in, so its device address is looked up here.
+bitnet_status noalloc_scratch(int dev, void **addr)
+{
+    if (!g_na_dev_addr[dev]) {
+        void *a = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_tmaps);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc tensor-map array)");
+        g_na_dev_addr[dev] = a;
+    }
+    *addr = g_na_dev_addr[dev];
+    return BITNET_OK;
+}
+
+// Same byte-balanced partition as the ordinary stack call, over fixed arrays.
+bitnet_status noalloc_plan_and_launch(int count, int m, int32_t *flags, cudaStream_t st, const DevInfo &dev,
+                                      const CUtensorMap *maps)
+{
+    GemvParams &p = g_na_params;
+    const LayerReq *L = g_na_layers;
+    int ninp = 0;
+    int64_t max_kpad = 0;
+    for (int i = 0; i < count; ++i) {
+        int found = -1;
+        for (int j = 0; j < ninp; ++j)
+            if (p.inp[j].x == L[i].x && p.inp[j].k == int32_t(L[i].w.k)) {
+                found = j;
+                break;
+            }
+        if (found < 0) {
+            found = ninp++;
+            p.inp[found].x = L[i].x;
+            p.inp[found].scale = nullptr;
+            p.inp[found].k = int32_t(L[i].w.k);
+            p.inp[found].kb = int32_t(blocks_of(L[i].w.k));
+        }
+        g_na_input_of[i] = found;
+        const int64_t kp = 128 * blocks_of(L[i].w.k);
+        if (kp > max_kpad) max_kpad = kp;
+        p.lin[i].tmap = maps + i;
+        p.lin[i].y = L[i].y;
+        p.lin[i].acc = L[i].acc;
+        p.lin[i].n = int32_t(L[i].w.n);
+        p.lin[i].kb = int32_t(blocks_of(L[i].w.k));
+        p.lin[i].scale = L[i].w.scale;
+        p.lin[i].input = found;
+    }
+    const int variant = pick_variant(m, max_kpad);
+    if (variant < 0)
+        return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: m=%d x kpad=%lld exceeds the GEMV activation area", m,
+                    (long long)max_kpad);
+    const int64_t xcap = x_cap(kVariants[variant].nw, kVariants[variant].boxes);
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) total += L[i].w.n * 32 * blocks_of(L[i].w.k);
+    const int64_t G = dev.sm_count;
+    int nr = 0, ns = 0, cur_target = -1;
+    int64_t cur_x = 0, xmax = 0, cum = 0;
+    bool open = false;
+    for (int i = 0; i < count; ++i) {
+        const int64_t rowb = 32 * blocks_of(L[i].w.k);
+        const int64_t tiles = (L[i].w.n + kTileRows - 1) / kTileRows;
+        const int64_t xin = int64_t(m) * 128 * blocks_of(L[i].w.k);
+        for (int64_t t = 0; t < tiles; ++t) {
+            const int64_t rows = (t + 1 < tiles) ? kTileRows : L[i].w.n - t * kTileRows;
+            const int64_t tb = rows * rowb;
+            const int target = int((cum + tb / 2) * G / total);
+            cum += tb;
+            if (open && target != cur_target) {
+                if (p.rng[nr].nseg > 0) {
+                    xmax = cur_x > xmax ? cur_x : xmax;
+                    ++nr;
+                }
+                open = false;
+            }
+            for (;;) {
+                if (!open) {
+                    if (nr == kMaxRanges) return fail(BITNET_ERR_INVALID_ARG, "noalloc stack needs more than %d CTAs", kMaxRanges);
+                    p.rng[nr].seg0 = int16_t(ns);
+                    p.rng[nr].nseg = 0;
+                    p.rng[nr].nin = 0;
+                    cur_x = 0;
+                    cur_target = target;
+                    open = true;
+                }
+                GemvRange &r = p.rng[nr];
+                int slot = -1;
+                for (int u = 0; u < r.nin; ++u)
+                    if (r.in[u] == g_na_input_of[i]) slot = u;
+                const bool same_seg = r.nseg > 0 && p.seg[ns - 1].lin == i && p.seg[ns - 1].tile1 == t;
+                const bool need_in = slot < 0;
+                if ((need_in && (r.nin == kMaxRangeInputs || cur_x + xin > xcap)) ||
+                    (!same_seg && (r.nseg == kMaxRangeSegs || ns == kMaxSegs))) {
+                    if (r.nseg == 0 || ns == kMaxSegs)
+                        return fail(BITNET_ERR_INVALID_ARG, "noalloc stack too large for one launch");
+                    xmax = cur_x > xmax ? cur_x : xmax;
+                    ++nr;
+                    open = false;
+                    continue;
+                }
+                if (need_in) {
+                    slot = r.nin;
+                    r.in[r.nin++] = int16_t(g_na_input_of[i]);
+                    cur_x += xin;
+                }
+                if (!same_seg) {
+                    GemvSeg &sg = p.seg[ns++];
+                    sg.lin = int16_t(i);
+                    sg.slot = int16_t(slot);
+                    sg.tile0 = int32_t(t);
+                    sg.tile1 = int32_t(t + 1);
+                    r.nseg++;
+                } else {
+                    p.seg[ns - 1].tile1 = int32_t(t + 1);
+                }
+                break;
+            }
+        }
+    }
+    if (open && p.rng[nr].nseg > 0) {
+        xmax = cur_x > xmax ? cur_x : xmax;
+        ++nr;
+    }
+    p.m = m;
+    p.num_ranges = nr;
+    p.prequant = 0;
+    p.force_stall = g_force_stall;
+    p.flags = flags;
+    p.wait_limit = wait_limit();
+    p.trace = g_trace;
+    p.x_bytes = int32_t((xmax + 127) / 128 * 128);
+    p.fence_maps = 1;   // the fixed array is rewritten in place between calls
+    cudaError_t e = launch_gemv(p, variant, st);
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemv launch");
+}
+
+}  // namespace
+
+extern "C" bitnet_status bitnet_linear_stack_noalloc(const float *const *x, int64_t m, const bitnet_tw *w,
+                                                     int64_t count, float *const *y, int32_t *const *acc_out,
+                                                     int32_t *d_flags, void *stream)
+{
+    if (!x || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: NULL array");
+    if (count < 1 || count > kNoallocMaxLayers)
+        return fail(BITNET_ERR_INVALID_ARG,
+                    "noalloc stack: count=%lld exceeds the %d tensor maps its fixed device array holds",
+                    (long long)count, kNoallocMaxLayers);
+    if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: bad m");
+    for (int64_t i = 0; i < count; ++i) {
+        bitnet_status s = check_tw(w[i], i);
+        if (s != BITNET_OK) return s;
+        if (!x[i] || !y[i])
+            return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: layer %lld has a NULL x or y", (long long)i);
+        if (!aligned(x[i], 16))
+            return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: layer %lld x not 16-byte aligned", (long long)i);
+    }
+    DevInfo dev;
+    bitnet_status s = check_device(&dev);
+    if (s != BITNET_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    std::lock_guard<std::mutex> lock(g_na_mu);
+    void *scratch = nullptr;
+    s = noalloc_scratch(dev.ordinal, &scratch);
+    if (s != BITNET_OK) return s;
+    const int n = int(count);
+    // rewrite the device array only when it does not already hold these maps
+    bool same = g_na_copied_count[dev.ordinal] == n;
+    for (int i = 0; same && i < n; ++i) {
+        const NaKey &k = g_na_copied[dev.ordinal][i];
+        same = k.p == w[i].packed && k.n == w[i].n && k.k == w[i].k;
+    }
+    if (!same) {
+        for (int i = 0; i < n; ++i) {
+            s = encode_weight_map(&g_na_host_maps[i], w[i].packed, w[i].n, blocks_of(w[i].k));
+            if (s != BITNET_OK) return s;
+        }
+        // from pageable memory: the bytes are staged before this returns, so
+        // the host array may be rewritten by the next call
+        cudaError_t e = cudaMemcpyAsync(scratch, g_na_host_maps, size_t(n) * sizeof(CUtensorMap),
+                                        cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) {
+            g_na_copied_count[dev.ordinal] = 0;
+            return cuda_fail(e, "noalloc tensor-map copy");
+        }
+        for (int i = 0; i < n; ++i) g_na_copied[dev.ordinal][i] = NaKey{w[i].packed, w[i].n, w[i].k};
+        g_na_copied_count[dev.ordinal] = n;
+    }
+    const CUtensorMap *maps = static_cast<const CUtensorMap *>(scratch);
+    for (int64_t m0 = 0; m0 < m; m0 += BITNET_GEMV_MAX_M) {
+        const int ms = int((m - m0) < BITNET_GEMV_MAX_M ? (m - m0) : BITNET_GEMV_MAX_M);
+        for (int i = 0; i < n; ++i) {
+            LayerReq &r = g_na_layers[i];
+            r.x = x[i] + m0 * w[i].k;
+            r.xscale = nullptr;
+            r.w = w[i];
+            r.y = y[i] + m0 * w[i].n;
+            r.acc = (acc_out && acc_out[i]) ? acc_out[i] + m0 * w[i].n : nullptr;
+        }
+        s = noalloc_plan_and_launch(n, ms, d_flags, st, dev, maps);
+        if (s != BITNET_OK) return s;
+    }
+    return BITNET_OK;
+}
