@@ -150,16 +150,18 @@ def build_stack(m, dev, layers=28):
     from ternary_weight_i2_b200 import synth
 
     packed, tws = [], []
+    fl = torch.zeros(1, dtype=torch.int32, device=dev)
     for L in range(layers):
         for (name, n, k), (w, s) in zip(synth.LAYER_SHAPES, synth.layer_weights(L, 3)):
             wt = torch.from_numpy(w).to(dev)
             pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
-            fl = torch.zeros(1, dtype=torch.int32, device=dev)
             tw2.pack_ternary(wt, pk, flags=fl)
             del wt
             packed.append(pk)
             tws.append(tw2.make_tw(pk, n, k, s))
     torch.cuda.synchronize()
+    if int(fl.item()) != 0:
+        raise RuntimeError("pack flagged a non-ternary weight")
     # all distinct inputs in one buffer, all outputs in another
     in_sizes = [m * k for _ in range(layers) for k in synth.LAYER_INPUT_K]
     out_sizes = [m * n for _ in range(layers) for (_, n, _) in synth.LAYER_SHAPES]
@@ -184,8 +186,10 @@ def build_stack(m, dev, layers=28):
     return packed, tws, xs, ys, x_host, x_dev, y_dev
 
 
-def time_device(call, steps, warmup, stream):
-    """Per-launch CUDA-event durations on `stream` and the whole-loop time."""
+def time_device(call, steps, warmup, stream, profile_range=False):
+    """Per-launch CUDA-event durations on `stream` and the whole-loop time.
+    With profile_range the timed loop is bracketed by cudaProfilerStart/Stop,
+    so that a profiler started with --profile-from-start off sees only it."""
     import torch
     for _ in range(warmup):
         call()
@@ -194,11 +198,15 @@ def time_device(call, steps, warmup, stream):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     _barrier()
     torch.cuda.synchronize()
+    if profile_range:
+        torch.cuda.cudart().cudaProfilerStart()
     for i in range(steps):
         starts[i].record(stream)
         call()
         ends[i].record(stream)
     torch.cuda.synchronize()
+    if profile_range:
+        torch.cuda.cudart().cudaProfilerStop()
     _barrier()
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total = starts[0].elapsed_time(ends[-1])
@@ -256,7 +264,7 @@ def run_gpu(args):
     for _ in range(int(args.soak / 1e-4)):   # untimed soak of the same launch before timing
         graph.replay()
     clocks.start()
-    total_ms, per = time_device(graph.replay, args.steps, args.warmup, stream)
+    total_ms, per = time_device(graph.replay, args.steps, args.warmup, stream, profile_range=True)
     clk = clocks.stop()
     if int(flags.item()) != 0:
         raise RuntimeError(f"device flags {int(flags.item())} during the timed run")
