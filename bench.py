@@ -49,6 +49,7 @@ def _args():
     ap.add_argument("--no-sweep", action="store_true", help="skip the M = 2, 4, 8 lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the M=2048 prefill GEMM line")
     ap.add_argument("--soak", type=float, default=0.5,
                     help="seconds of untimed launches before timing (clock sampling window)")
     ap.add_argument("--layers", type=int, default=28,
@@ -315,6 +316,10 @@ def run_gpu(args):
             sweep[str(ms)] = {"tokens_per_s": round(world * ms / (t2 / 50 * 1e-3), 1),
                               "weight_gbs": round(stack_bytes / (k2 * 1e-3) / 1e9, 1)}
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill(dev, stream, flags, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(budget_s=12.0)
@@ -339,10 +344,80 @@ def run_gpu(args):
             "gpu_launches": args.steps,
             "clocks": clk,
             "m_sweep": sweep,
+            "prefill": prefill,
         }
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+PREFILL_M = 2048
+PREFILL_OPS = 2 * PREFILL_M * sum(n * k for _, n, k in
+                                  [("q", 1536, 1536), ("k", 256, 1536), ("v", 256, 1536), ("o", 1536, 1536),
+                                   ("gate", 8960, 1536), ("up", 8960, 1536), ("down", 1536, 8960)])
+
+
+def run_prefill(dev, stream, flags, world):
+    """M=2048 prefill over the seven decoder-layer shapes: int8 activations
+    pre-quantised by bitnet_quant_act (timed separately), then seven
+    bitnet_linear_q launches (the tcgen05 GEMM) per step, graph-replayed."""
+    import torch
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import synth
+
+    xs = synth.prefill_inputs(PREFILL_M)
+    xq, xs_scale, x_dev = {}, {}, {}
+    for k, x in xs.items():
+        x_dev[k] = torch.from_numpy(x).to(dev)
+        xq[k] = torch.empty((PREFILL_M, tw2.kpad(k)), dtype=torch.int8, device=dev)
+        xs_scale[k] = torch.empty(PREFILL_M, dtype=torch.float32, device=dev)
+    tws, ys, keep = [], [], []
+    for i, (name, n, k) in enumerate(synth.LAYER_SHAPES):
+        rng = np.random.default_rng(synth.seed_for(4, i))
+        w = synth.ternary(rng, n, k)
+        s = synth.weight_scale(rng)
+        pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
+        tw2.pack_ternary(torch.from_numpy(w).to(dev), pk, flags=flags)
+        keep.append(pk)
+        tws.append((name, n, k, tw2.make_tw(pk, n, k, s)))
+        ys.append(torch.empty((PREFILL_M, n), dtype=torch.float32, device=dev))
+
+    def quant():
+        for k in xs:
+            tw2.quant_act(x_dev[k], xq[k], xs_scale[k], flags=flags)
+
+    def gemms():
+        for (name, n, k, tw), y in zip(tws, ys):
+            tw2.linear_q(xq[k], xs_scale[k], tw, y, flags=flags)
+
+    quant()
+    gemms()
+    torch.cuda.synchronize()
+    gq, gg = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gq):
+        quant()
+    with torch.cuda.graph(gg):
+        gemms()
+    tq, _ = time_device(gq.replay, 20, 3, stream)
+    tg, per = time_device(gg.replay, 20, 3, stream)
+    tq, tg = _max_over_ranks(tq) / 20, _max_over_ranks(tg) / 20
+    per_shape = {}
+    for (name, n, k, tw), y in zip(tws, ys):
+        t, _ = time_device(lambda: tw2.linear_q(xq[k], xs_scale[k], tw, y, flags=flags), 10, 2, stream)
+        per_shape[name] = {"ms": round(t / 10, 5), "tops": round(2 * PREFILL_M * n * k / (t / 10 * 1e-3) / 1e12, 1)}
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"device flags {int(flags.item())} in the prefill run")
+    _, _, peaks = _peaks()
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    peak = 2.0 * bf16          # int8 dense = 2 x bf16 dense (nominal 4.5 vs 2.25 PFLOP/s)
+    tops = world * PREFILL_OPS / (tg * 1e-3) / 1e12
+    return {"workload": "M=2048 tokens x the seven decoder-layer shapes, int8 activations x ternary weights",
+            "ops_per_step": PREFILL_OPS, "ms_per_step": round(tg, 5), "tops": round(tops, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tops / world, 1), "peak": round(peak, 1),
+                         "unit": "TOPS", "frac": round(tops / world / peak, 4),
+                         "peak_kind": "measured bf16 cuBLAS burst (MEASURED_PEAKS.json) x 2 (int8:bf16 dense ratio)"},
+            "quant_ms_per_step": round(tq, 5), "per_shape": per_shape,
+            "kernel": "gemm_i2_kernel (tcgen05.mma kind::i8, 128x256x128 tiles)"}
 
 
 def build_stack_views(m, dev, tws, layers=28):

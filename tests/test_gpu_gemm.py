@@ -1,0 +1,95 @@
+"""Parity of the prefill path (M > 8: per-token quantiser + tcgen05 int8 GEMM)
+with the CPU oracle, through the C ABI.  Full comparisons on shapes the oracle
+finishes in seconds (several 128 x 256 tiles and ragged tails); at the prefill
+size (M = 2048 over the seven decoder-layer shapes, the launch bench.py times)
+every output is checked against its exact int32 sum by the dequantisation
+identity and sampled output columns against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ternary_weight_i2_b200 as tw2
+from ternary_weight_i2_b200 import synth
+
+from gpu_helpers import DEV, Guarded, flags_tensor, pack_on_gpu, rel_err, upload
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+
+def _run(x, w, s_w, quantised=False):
+    m, k = x.shape
+    n = w.shape[0]
+    pk = pack_on_gpu(w)
+    tw = tw2.make_tw(pk, n, k, s_w)
+    y = Guarded((m, n), torch.float32)
+    acc = Guarded((m, n), torch.int32)
+    fl = flags_tensor()
+    if quantised:
+        q, s_act, _ = oracle.quant_act(x)
+        tw2.linear_q(upload(q), upload(s_act), tw, y.t, acc=acc.t, flags=fl)
+    else:
+        ws = torch.empty(tw2.linear_workspace_bytes(m, k), dtype=torch.uint8, device=DEV)
+        tw2.linear(upload(x), tw, y.t, acc=acc.t, workspace=ws, flags=fl)
+    torch.cuda.synchronize()
+    assert int(fl.item()) == 0
+    assert y.guard_intact() and acc.guard_intact()
+    return y.t.cpu().numpy(), acc.t.cpu().numpy()
+
+
+@pytest.mark.parametrize("m,k,n", [(9, 128, 256), (128, 128, 256), (128, 1536, 256), (130, 1536, 300),
+                                   (257, 1536, 512), (300, 9024, 264), (2048, 1536, 256)])
+@pytest.mark.parametrize("quantised", [False, True])
+def test_gemm_full_parity(m, k, n, quantised):
+    rng = np.random.default_rng(m * 7 + k + n)
+    w = synth.ternary(rng, n, k)
+    x = synth.normal_row_spread(rng, m, k)
+    s_w = synth.weight_scale(rng)
+    yg, ag = _run(x, w, s_w, quantised)
+    pk_np, _ = oracle.pack(w)
+    a_want, y64, y32, st = oracle.linear(x, pk_np, n, k, s_w)
+    assert st == 0
+    np.testing.assert_array_equal(ag, a_want)
+    assert rel_err(yg, y64) <= RTOL
+    np.testing.assert_array_equal(yg.view(np.uint32), y32.view(np.uint32))
+
+
+def test_gemm_special_rows_and_saturation():
+    m, k, n = 200, 9024, 256
+    x = np.full((m, k), 0.25, np.float32)
+    x[1] = -0.25
+    x[2] = 0.0
+    x[3, 5] = np.float32(3e4)
+    w = np.ones((n, k), np.int8)
+    w[1] = -1
+    w[2] = 0
+    w[3::2] = synth.ternary(np.random.default_rng(1), (n - 3 + 1) // 2, k)
+    yg, ag = _run(x, w, 0.03)
+    pk_np, _ = oracle.pack(w)
+    a_want, _, y32, _ = oracle.linear(x, pk_np, n, k, 0.03)
+    np.testing.assert_array_equal(ag, a_want)
+    np.testing.assert_array_equal(yg.view(np.uint32), y32.view(np.uint32))
+    assert ag[0, 0] == 127 * 9024 and ag[1, 0] == -127 * 9024 and ag[0, 1] == -127 * 9024
+
+
+@pytest.mark.parametrize("shape", range(len(synth.LAYER_SHAPES)))
+def test_prefill_2048_sampled(shape):
+    name, n, k = synth.LAYER_SHAPES[shape]
+    rng = np.random.default_rng(synth.seed_for(4, shape))
+    w = synth.ternary(rng, n, k)
+    s_w = synth.weight_scale(rng)
+    x = synth.prefill_inputs(2048)[k]
+    yg, ag = _run(x, w, s_w)
+    cols = np.unique(np.concatenate([[0, 1, 255, min(256, n - 1), n - 1], rng.choice(n, 11, replace=False)]))
+    pk_np, _ = oracle.pack(w[cols])
+    a_want, y64, y32, _ = oracle.linear(x, pk_np, len(cols), k, s_w)
+    np.testing.assert_array_equal(ag[:, cols], a_want)
+    np.testing.assert_array_equal(yg[:, cols].view(np.uint32), y32.view(np.uint32))
+    # every output is the dequantisation of its own accumulator
+    _, s_act, _ = oracle.quant_act(x)
+    y_all = (ag.astype(np.float32) * s_act[:, None]).astype(np.float32) * np.float32(s_w)
+    np.testing.assert_array_equal(yg.view(np.uint32), y_all.view(np.uint32))
+    # |acc| is bounded by sum_k |q| for ternary weights
+    q, _, _ = oracle.quant_act(x)
+    assert (np.abs(ag.astype(np.int64)) <= np.abs(q.astype(np.int64)).sum(axis=1)[:, None]).all()
