@@ -50,6 +50,8 @@ def _args():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the M=2048 prefill GEMM line")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the M=2048 prefill GEMMs (profiling aid) and print their object")
     ap.add_argument("--soak", type=float, default=0.5,
                     help="seconds of untimed launches before timing (clock sampling window)")
     ap.add_argument("--layers", type=int, default=28,
@@ -403,7 +405,10 @@ def run_prefill(dev, stream, flags, world):
     tq, tg = _max_over_ranks(tq) / 20, _max_over_ranks(tg) / 20
     per_shape = {}
     for (name, n, k, tw), y in zip(tws, ys):
-        t, _ = time_device(lambda: tw2.linear_q(xq[k], xs_scale[k], tw, y, flags=flags), 10, 2, stream)
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1):
+            tw2.linear_q(xq[k], xs_scale[k], tw, y, flags=flags)
+        t, _ = time_device(g1.replay, 10, 2, stream)
         per_shape[name] = {"ms": round(t / 10, 5), "tops": round(2 * PREFILL_M * n * k / (t / 10 * 1e-3) / 1e12, 1)}
     if int(flags.item()) != 0:
         raise RuntimeError(f"device flags {int(flags.item())} in the prefill run")
@@ -509,6 +514,16 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.prefill_only:
+        import torch
+        import ternary_weight_i2_b200 as tw2
+        from ternary_weight_i2_b200 import build as tbuild
+        tbuild.build()
+        tw2.load()
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        flags = torch.zeros(1, dtype=torch.int32, device=dev)
+        print(json.dumps(run_prefill(dev, torch.cuda.current_stream(), flags, 1)))
     else:
         run_gpu(args)
 

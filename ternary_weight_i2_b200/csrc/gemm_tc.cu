@@ -15,15 +15,19 @@
 // K block (one packed block per weight row):
 //   warp 0      TMA: the activation tile (128 rows x 128 B, 128-byte swizzle,
 //               the canonical K-major layout of the MMA) and the packed weight
-//               tile (256 rows x 32 B) into a 3-stage shared-memory ring;
-//   warps 2-3   expand the packed tile to signed int8 (code - 1) straight into
-//               the canonical K-major 128-byte-swizzled layout of operand B;
-//   warp 1      one thread issues 4 tcgen05.mma (M=128, N=256, K=32) per
-//               block into a TMEM accumulator (two 256-column accumulators,
-//               so the epilogue of one tile overlaps the next tile's K loop)
-//               and commits to mbarriers;
-//   warps 4-7   epilogue: tcgen05.ld the accumulator (one TMEM lane = one
-//               output row per thread), dequantise in fp32, store.
+//               tile (256 rows x 32 B) into a 6-stage shared-memory ring;
+//   warps 3-6   expand the packed tile into the canonical K-major
+//               128-byte-swizzled layout of operand B (two buffers), as the
+//               unsigned codes w + 1 in {0, 1, 2}: one mask per 2-bit field;
+//   warp 2      sums each activation row of the tile (sum_k q), so that the
+//               epilogue can remove the +1 of the codes: acc = D - sum_k q;
+//   warp 1      one thread issues 4 tcgen05.mma (M=128, N=256, K=32, signed A
+//               x unsigned B) per block into a TMEM accumulator (two 256-column
+//               accumulators, so the epilogue of one tile overlaps the next
+//               tile's K loop) and commits to mbarriers;
+//   warps 7-10  epilogue: tcgen05.ld the accumulator (one TMEM lane = one
+//               output row per thread), subtract the row sum, dequantise in
+//               fp32, store.
 // Every wait is bounded; on expiry the CTA raises BITNET_FLAG_TIMEOUT, the
 // other roles stop, in-flight copies and MMAs are drained (bounded) and TMEM
 // is freed before exit.  No TMA multicast.
@@ -35,20 +39,26 @@
 namespace bitnet {
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 5;                         // TMA ring (activations + packed weights)
+constexpr int kBBufs = 2;                          // expanded weight tiles
 constexpr int kAStage = kBM * kBK;                 // 16 KB int8 activations
-constexpr int kBStage = kBN * kBK;                 // 32 KB expanded int8 weights
+constexpr int kBStage = kBN * kBK;                 // 32 KB expanded weight codes
 constexpr int kPStage = kBN * 32;                  // 8 KB packed weights
-constexpr int kStageBytes = kAStage + kBStage + kPStage;
-constexpr int kGemmThreads = 256;
-constexpr int kExpandThreads = 64;                 // warps 2-3
-constexpr int kEpiThreads = 128;                   // warps 4-7
+constexpr int kStageOut = 32 * 128;                // one 32 x 32 fp32 output chunk (128-byte rows)
+constexpr int kAOff = 0, kPOff = kStages * kAStage, kBOff = kPOff + kStages * kPStage;
+constexpr int kOOff = kBOff + 2 * kBStage;         // 4 epilogue warps x 2 output staging buffers
+constexpr int kGemmThreads = 352;                  // 11 warps
+constexpr int kExpandWarp0 = 3, kExpandWarps = 4, kExpandThreads = 32 * kExpandWarps;
+constexpr int kEpiWarp0 = 7, kEpiThreads = 128;
 constexpr int kTmemCols = 2 * kBN;                 // two int32 accumulators
-constexpr int kGemmSmem = 1024 + kStages * kStageBytes;
+constexpr int kGemmSmem = 1024 + kOOff + 4 * 2 * kStageOut;
 
 struct GemmParams {
     CUtensorMap tmap_a;       // int8 q [M, Kpad]: dims {Kpad, M}, box {128, 128}, 128-byte swizzle
     CUtensorMap tmap_b;       // packed [N, 32*KB]: dims {32*KB, N}, box {32, 256}, no swizzle
+    CUtensorMap tmap_y;       // fp32 y [M, N]: dims {N, M}, box {32, 32}, 128-byte swizzle (when tma_out)
+    CUtensorMap tmap_acc;     // int32 acc [M, N], same shape (when tma_out and acc)
+    int32_t tma_out;          // outputs through TMA stores (N % 4 == 0), else direct stores
     const float *act_scale;   // [M]
     float *y;                 // [M, N]
     int32_t *acc;             // [M, N] or null
@@ -57,7 +67,15 @@ struct GemmParams {
     int32_t tiles_m, tiles_n;
     int32_t *flags;
     uint64_t wait_limit;
+    uint64_t *trace;          // optional: CTA 0 per-K-block globaltimer stamps (kGemmTraceBlocks x 8)
 };
+
+// Trace of CTA 0 (profiling aid), per K block it < kGemmTraceBlocks:
+// [it*8 + 0] producer issued, 1 MMA saw full, 2 MMA saw B ready, 3 MMA issued,
+// 4 expander saw full, 5 expander saw B free, 6 expander done, 7 row sums done;
+// then [kGemmTraceBlocks*8 + 0] kernel entry, +1 set-up done, +2 all roles
+// done, +8+t epilogue of the CTA's tile t (t < 8) done.
+constexpr int kGemmTraceBlocks = 64;
 
 // ------------------------------------------------------------ tcgen05 PTX
 
@@ -76,9 +94,9 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
     return d;
 }
 
-// Instruction descriptor: kind::i8, D int32, A and B signed int8, both
-// K-major, M = 128, N = 256, dense.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+// Instruction descriptor: kind::i8, D int32, A signed int8, B unsigned int8,
+// both K-major, M = 128, N = 256, dense.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (0u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
 {
@@ -95,6 +113,21 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// 2-D TMA store of a shared-memory box to global memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src, int32_t x, int32_t y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap), "r"(x),
+                 "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
@@ -109,12 +142,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Signed int8 weights (code - 1) of field g of a packed word: one byte per
-// element, elements 32g + b .. 32g + b + 3 of the block.
+// Codes w + 1 of field g of a packed word as unsigned bytes: elements
+// 32g + b .. 32g + b + 3 of the block.
 __device__ __forceinline__ uint32_t expand_field(uint32_t v, int g)
 {
-    const uint32_t c = (v >> (2 * g)) & 0x03030303u;   // codes 0, 1, 2 per byte
-    return (c + 0x7F7F7F7Fu) ^ 0x80808080u;            // 0x7F+c has no carry; ^0x80 -> c - 1
+    return (v >> (2 * g)) & 0x03030303u;
 }
 
 // Wait on an mbarrier phase; false on timeout or when another role aborted.
@@ -133,8 +165,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    __shared__ __align__(8) uint64_t full_bar[kStages], expd_bar[kStages], empty_bar[kStages];
+    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+    __shared__ __align__(8) uint64_t bready_bar[kBBufs], bfree_bar[kBBufs];
     __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
+    __shared__ int32_t rowsum[2][kBM];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     volatile int *abort_flag = &abort_s;
@@ -143,15 +177,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
     const uint64_t limit = p.wait_limit;
     const int ntiles = p.tiles_m * p.tiles_n;
     const int kblocks = p.kb;
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *ctrace = (p.trace && blockIdx.x == 0) ? p.trace + kGemmTraceBlocks * 8 : nullptr;
+    if (ctrace && tid == 0) ctrace[0] = globaltimer();
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
-            mbar_init(smem_u32(&expd_bar[s]), kExpandThreads);
-            mbar_init(smem_u32(&empty_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1 + kExpandWarps + 1);   // MMA, expanders, row sums
+        }
+        for (int b = 0; b < kBBufs; ++b) {
+            mbar_init(smem_u32(&bready_bar[b]), kExpandThreads);
+            mbar_init(smem_u32(&bfree_bar[b]), 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&accf_bar[b]), 1);
+            mbar_init(smem_u32(&accf_bar[b]), 2);                       // MMA, row sums
             mbar_init(smem_u32(&acce_bar[b]), kEpiThreads);
         }
         mbar_init(smem_u32(&drain_bar), 1);
@@ -168,17 +208,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_s;
+    if (ctrace && tid == 0) ctrace[1] = globaltimer();
 
     auto fail = [&]() {
         abort_s = 1;
         raise_flag(p.flags, BITNET_FLAG_TIMEOUT);
+    };
+    uint64_t *trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
+    auto stamp = [&](int it, int ev) {
+        if (trace && it < kGemmTraceBlocks) trace[it * 8 + ev] = globaltimer();
     };
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_w = l2_evict_first_policy();
-            int it = 0, issued_tail = 0;
+            int it = 0, last = -1;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 const int m_tile = t % p.tiles_m, n_tile = t / p.tiles_m;
@@ -189,23 +234,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                         ok = false;
                         break;
                     }
-                    uint8_t *st = smem + s * kStageBytes;
                     const uint32_t fb = smem_u32(&full_bar[s]);
                     mbar_arrive_expect_tx(fb, kAStage + kPStage);
                     asm volatile(
                         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(st)),
+                        " [%0], [%1, {%2, %3}], [%4];" ::"r"(sbase + kAOff + s * kAStage),
                         "l"(&p.tmap_a), "r"(kb * kBK), "r"(m_tile * kBM), "r"(fb)
                         : "memory");
-                    tma_load_2d(smem_u32(st + kAStage + kBStage), &p.tmap_b, kb * 32, n_tile * kBN, fb, pol_w);
-                    issued_tail = it;
+                    tma_load_2d(sbase + kPOff + s * kPStage, &p.tmap_b, kb * 32, n_tile * kBN, fb, pol_w);
+                    stamp(it, 0);
+                    last = it;
                 }
             }
-            if (!ok) {
-                // let copies already issued land before the CTA can exit
-                for (int j = (issued_tail >= kStages ? issued_tail - kStages + 1 : 0); j <= issued_tail; ++j)
+            if (!ok)   // let copies already issued land before the CTA can exit
+                for (int j = (last >= kStages ? last - kStages + 1 : 0); j <= last; ++j)
                     mbar_wait(smem_u32(&full_bar[j % kStages]), (j / kStages) & 1, kDrainWaitLimit);
-            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
@@ -223,20 +266,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                 const uint32_t d_tmem = tmem_base + uint32_t(b * kBN);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int s = it % kStages, r = it / kStages;
-                    if (!wait_or_abort(smem_u32(&full_bar[s]), r & 1, limit, abort_flag) ||
-                        !wait_or_abort(smem_u32(&expd_bar[s]), r & 1, limit, abort_flag)) {
+                    const int bb = it % kBBufs, rb = it / kBBufs;
+                    const bool f1 = wait_or_abort(smem_u32(&full_bar[s]), r & 1, limit, abort_flag);
+                    stamp(it, 1);
+                    if (!f1 || !wait_or_abort(smem_u32(&bready_bar[bb]), rb & 1, limit, abort_flag)) {
                         fail();
                         ok = false;
                         break;
                     }
+                    stamp(it, 2);
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + s * kStageBytes);
-                    const uint32_t b0 = a0 + kAStage;
+                    const uint32_t a0 = sbase + kAOff + s * kAStage;
+                    const uint32_t b0 = sbase + kBOff + bb * kBStage;
 #pragma unroll
                     for (int ks = 0; ks < kBK / 32; ++ks)
                         mma_i8(d_tmem, sw128_desc(a0 + ks * 32), sw128_desc(b0 + ks * 32),
                                (kb > 0 || ks > 0) ? 1u : 0u);
                     mma_commit(smem_u32(&empty_bar[s]));
+                    mma_commit(smem_u32(&bfree_bar[bb]));
+                    stamp(it, 3);
                     any = true;
                 }
                 if (ok) mma_commit(smem_u32(&accf_bar[b]));
@@ -247,24 +295,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                 mbar_wait(smem_u32(&drain_bar), 0, kDrainWaitLimit);
             }
         }
-    } else if (warp < 4) {
+    } else if (warp == 2) {
+        // -------------------------------------------- activation row sums
+        // lane = (row group rg = lane/8, 16-byte chunk c = lane%8); rows 4i+rg
+        const int c = lane & 7, rg = lane >> 3;
+        int it = 0, tcount = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+            const int b = tcount & 1, ur = tcount >> 1;
+            int32_t ps[kBM / 4];
+#pragma unroll
+            for (int i = 0; i < kBM / 4; ++i) ps[i] = 0;
+            for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                const int s = it % kStages, r = it / kStages;
+                const bool landed = wait_or_abort(smem_u32(&full_bar[s]), r & 1, limit, abort_flag);
+                if (!__all_sync(0xffffffffu, landed)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                const uint32_t a0 = sbase + kAOff + s * kAStage;
+#pragma unroll
+                for (int i = 0; i < kBM / 4; ++i) {
+                    const uint4 v = lds128(a0 + (4 * i + rg) * 128 + c * 16);
+                    int32_t acc = ps[i];
+                    asm("dp4a.s32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(v.x), "r"(0x01010101));
+                    asm("dp4a.s32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(v.y), "r"(0x01010101));
+                    asm("dp4a.s32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(v.z), "r"(0x01010101));
+                    asm("dp4a.s32.s32 %0, %1, %2, %0;" : "+r"(acc) : "r"(v.w), "r"(0x01010101));
+                    ps[i] = acc;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&empty_bar[s]));
+                    stamp(it, 7);
+                }
+            }
+            if (!ok) break;
+            if (ur > 0) {
+                const bool freed = wait_or_abort(smem_u32(&acce_bar[b]), (ur - 1) & 1, limit, abort_flag);
+                if (!__all_sync(0xffffffffu, freed)) {
+                    if (lane == 0) fail();
+                    break;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kBM / 4; ++i) {
+                int32_t v = ps[i];
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                if (c == 0) rowsum[b][4 * i + rg] = v;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&accf_bar[b]));
+        }
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------- expanders
-        const int et = tid - 64;
+        const int et = tid - 32 * kExpandWarp0;
         int it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int s = it % kStages, r = it / kStages;
-                const bool landed = wait_or_abort(smem_u32(&full_bar[s]), r & 1, limit, abort_flag);
-                if (!landed) {
-                    fail();
+                const int bb = it % kBBufs, rb = it / kBBufs;
+                bool go = wait_or_abort(smem_u32(&full_bar[s]), r & 1, limit, abort_flag);
+                if (et == 0) stamp(it, 4);
+                if (go && rb > 0) go = wait_or_abort(smem_u32(&bfree_bar[bb]), (rb - 1) & 1, limit, abort_flag);
+                if (et == 0) stamp(it, 5);
+                if (!__all_sync(0xffffffffu, go)) {
+                    if (lane == 0) fail();
                     ok = false;
                     break;
                 }
-                uint8_t *st = smem + s * kStageBytes;
-                const uint32_t bsm = smem_u32(st + kAStage);
-                const uint32_t psm = smem_u32(st + kAStage + kBStage);
-#pragma unroll 2
+                const uint32_t bsm = sbase + kBOff + bb * kBStage;
+                const uint32_t psm = sbase + kPOff + s * kPStage;
+#pragma unroll
                 for (int i = 0; i < (kBN * 2) / kExpandThreads; ++i) {
                     // task q: 8 consecutive rows with the same quad per quarter-warp
                     const int q = et + kExpandThreads * i;
@@ -282,68 +388,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                 }
                 // generic-proxy writes -> visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(smem_u32(&expd_bar[s]));
+                mbar_arrive(smem_u32(&bready_bar[bb]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));   // packed tile consumed
+                if (et == 0) stamp(it, 6);
             }
         }
     } else {
         // -------------------------------------------------------- epilogue
         const int sub = warp & 3;            // TMEM lanes 32*sub .. 32*sub+31
-        int tcount = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+        const uint32_t stage0 = sbase + kOOff + uint32_t(sub) * 2 * kStageOut;
+        int tcount = 0, chunk_no = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
             const int m_tile = t % p.tiles_m, n_tile = t / p.tiles_m;
             const int b = tcount & 1, ur = tcount >> 1;
             const bool ready = wait_or_abort(smem_u32(&accf_bar[b]), ur & 1, limit, abort_flag);
             if (!__all_sync(0xffffffffu, ready)) {
                 if (lane == 0) fail();
-                ok = false;
                 break;
             }
             tc_fence_after();
-            const int row = m_tile * kBM + 32 * sub + lane;
+            const int rloc = 32 * sub + lane;
+            const int row = m_tile * kBM + rloc;
             const bool row_ok = row < p.m;
             const float sa = row_ok ? p.act_scale[row] : 0.f;
+            const int32_t rs = rowsum[b][rloc];
             const uint32_t taddr = tmem_base + (uint32_t(32 * sub) << 16) + uint32_t(b * kBN);
-            const bool vec = (p.n % 4) == 0;
 #pragma unroll 1
             for (int c0 = 0; c0 < kBN; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(taddr + uint32_t(c0), v);
                 const int col0 = n_tile * kBN + c0;
-                if (!row_ok || col0 >= p.n) continue;
-                float *yr = p.y + size_t(row) * size_t(p.n) + col0;
-                int32_t *ar = p.acc ? p.acc + size_t(row) * size_t(p.n) + col0 : nullptr;
-                if (vec && col0 + 32 <= p.n) {
+                if (col0 >= p.n) continue;
+                if (p.tma_out) {
+                    // stage the 32 x 32 chunk (row = lane) in the 128-byte swizzled
+                    // layout and store it with one TMA store; tails are clipped by
+                    // the tensor map
+                    const uint32_t stg = stage0 + uint32_t(chunk_no & 1) * kStageOut;
+                    if (lane == 0) bulk_wait_read<1>();   // the store that used this buffer has read it
+                    __syncwarp();
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 o;
-                        o.x = __fmul_rn(__fmul_rn(float(int32_t(v[j + 0])), sa), p.w_scale);
-                        o.y = __fmul_rn(__fmul_rn(float(int32_t(v[j + 1])), sa), p.w_scale);
-                        o.z = __fmul_rn(__fmul_rn(float(int32_t(v[j + 2])), sa), p.w_scale);
-                        o.w = __fmul_rn(__fmul_rn(float(int32_t(v[j + 3])), sa), p.w_scale);
-                        *reinterpret_cast<float4 *>(yr + j) = o;
-                        if (ar)
-                            *reinterpret_cast<int4 *>(ar + j) =
-                                make_int4(int32_t(v[j]), int32_t(v[j + 1]), int32_t(v[j + 2]), int32_t(v[j + 3]));
+                    for (int j = 0; j < 8; ++j) {
+                        const int32_t a0 = int32_t(v[4 * j + 0]) - rs, a1 = int32_t(v[4 * j + 1]) - rs;
+                        const int32_t a2 = int32_t(v[4 * j + 2]) - rs, a3 = int32_t(v[4 * j + 3]) - rs;
+                        const uint32_t dst = stg + uint32_t(lane) * 128 + (uint32_t(j ^ (lane & 7)) << 4);
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                     "f"(__fmul_rn(__fmul_rn(float(a0), sa), p.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a1), sa), p.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a2), sa), p.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a3), sa), p.w_scale))
+                                     : "memory");
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&p.tmap_y, stg, col0, m_tile * kBM + 32 * sub);
+                        bulk_commit();
+                    }
+                    ++chunk_no;
+                    if (p.acc) {
+                        const uint32_t stg2 = stage0 + uint32_t(chunk_no & 1) * kStageOut;
+                        if (lane == 0) bulk_wait_read<1>();
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t dst = stg2 + uint32_t(lane) * 128 + (uint32_t(j ^ (lane & 7)) << 4);
+                            asm volatile("st.shared.v4.s32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                         "r"(int32_t(v[4 * j + 0]) - rs), "r"(int32_t(v[4 * j + 1]) - rs),
+                                         "r"(int32_t(v[4 * j + 2]) - rs), "r"(int32_t(v[4 * j + 3]) - rs)
+                                         : "memory");
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tmap_acc, stg2, col0, m_tile * kBM + 32 * sub);
+                            bulk_commit();
+                        }
+                        ++chunk_no;
                     }
                 } else {
+                    if (!row_ok) continue;
+                    float *yr = p.y + size_t(row) * size_t(p.n) + col0;
+                    int32_t *ar = p.acc ? p.acc + size_t(row) * size_t(p.n) + col0 : nullptr;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         if (col0 + j < p.n) {
-                            yr[j] = __fmul_rn(__fmul_rn(float(int32_t(v[j])), sa), p.w_scale);
-                            if (ar) ar[j] = int32_t(v[j]);
+                            const int32_t a = int32_t(v[j]) - rs;
+                            yr[j] = __fmul_rn(__fmul_rn(float(a), sa), p.w_scale);
+                            if (ar) ar[j] = a;
                         }
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&acce_bar[b]));
+            if (ctrace && tid == 32 * kEpiWarp0 && tcount < 8) ctrace[8 + tcount] = globaltimer();
         }
+        if (lane == 0) bulk_wait_all();   // every output store has completed
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (ctrace && tid == 0) ctrace[2] = globaltimer();
     if (warp == 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
@@ -367,7 +514,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn()
 bool gemm_available() { return true; }
 
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, cudaStream_t st)
+                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace,
+                        cudaStream_t st)
 {
     auto enc = gemm_encode_fn();
     if (!enc) return cudaErrorNotSupported;
@@ -393,6 +541,21 @@ cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, con
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    p.tma_out = (w->n % 4 == 0) ? 1 : 0;
+    if (p.tma_out) {
+        const cuuint64_t dims[2] = {cuuint64_t(w->n), cuuint64_t(m)};
+        const cuuint64_t strides[1] = {cuuint64_t(w->n) * 4};
+        const cuuint32_t box[2] = {32u, 32u};
+        const cuuint32_t es[2] = {1u, 1u};
+        if (enc(&p.tmap_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        if (acc && enc(&p.tmap_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, acc, dims, strides, box, es,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     p.act_scale = act_scale;
     p.y = y;
     p.acc = acc;
@@ -404,6 +567,7 @@ cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, con
     p.tiles_n = int32_t((w->n + kBN - 1) / kBN);
     p.flags = flags;
     p.wait_limit = wait_limit;
+    p.trace = trace;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(gemm_i2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
