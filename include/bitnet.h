@@ -104,6 +104,8 @@ typedef struct {
 #define BITNET_GEMV_MAX_M 8
 /* Largest number of layers one bitnet_linear_stack call takes. */
 #define BITNET_STACK_MAX 256
+/* Largest number of layers one bitnet_linear_q_grouped call takes. */
+#define BITNET_GROUP_MAX 8
 
 /* Library version as 10000*major + 100*minor + patch. */
 BITNET_API int bitnet_version(void);
@@ -185,6 +187,24 @@ BITNET_API bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_t
 BITNET_API bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t m,
                               const bitnet_tw *w, float *y, int32_t *acc_out,
                               int32_t *d_flags, void *stream);
+
+/*
+ * `count` independent layers on pre-quantised activations in one launch
+ * (prefill: the token count m is shared, each layer has its own input, weight
+ * and output; TR §3.2, Figure 6a).  m > 8 runs one persistent tensor-core GEMM
+ * over all layers' 128 x 256 output tiles, dealt to the SMs heaviest first, so
+ * that layers of different K and N balance inside one launch; m <= 8 runs the
+ * streaming GEMV.
+ *   xq[i]        device int8 [m, bitnet_kpad(w[i].k)], 16-byte aligned, pads 0
+ *   act_scale[i] device fp32 [m]
+ *   y[i]         device fp32 [m, w[i].n], 16-byte aligned
+ *   acc_out      NULL or host array of `count` device int32 [m, w[i].n] (entries
+ *                may be NULL)
+ * 1 <= count <= BITNET_GROUP_MAX.  Inputs may be shared between layers.
+ */
+BITNET_API bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                                 const bitnet_tw *w, int64_t count, float *const *y,
+                                                 int32_t *const *acc_out, int32_t *d_flags, void *stream);
 
 /*
  * A sequence of `count` independent ternary linear layers sharing the token

@@ -6,7 +6,7 @@ used by callers for device memory and streams.
 """
 from ._abi import (  # noqa: F401
     BitnetError, StackCall, TW, header_functions, kpad, linear, linear_q, linear_stack,
-    linear_stack_noalloc,
+    linear_stack_noalloc, linear_q_grouped, GroupedCall,
     linear_workspace_bytes, load, make_tw, pack_ternary, packed_bytes, quant_act,
     status_from_flags, unpack_ternary, version,
     FLAG_NONFINITE, FLAG_NOT_TERNARY, FLAG_TIMEOUT, GEMV_MAX_M, MAX_K, STACK_MAX,

@@ -49,6 +49,7 @@ _SIGNATURES = {
     "bitnet_linear": ([_P, _I64, C.POINTER(TW), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
     "bitnet_linear_q": ([_P, _P, _I64, C.POINTER(TW), _P, _P, _P, _P], C.c_int),
     "bitnet_linear_stack": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
+    "bitnet_linear_q_grouped": ([_P, _P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_linear_stack_noalloc": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
@@ -179,6 +180,32 @@ def linear_q(xq, act_scale, tw: TW, y, acc=None, flags=None, stream=None) -> Non
     m = xq.shape[0]
     _check(load().bitnet_linear_q(_ptr(xq), _ptr(act_scale), m, C.byref(tw), _ptr(y), _ptr(acc),
                                   _ptr(flags), _stream(stream)), "bitnet_linear_q")
+
+
+class GroupedCall:
+    """Marshalled arguments of one bitnet_linear_q_grouped call (reusable)."""
+
+    def __init__(self, xqs, scales, tws, ys, accs=None):
+        count = len(tws)
+        self.count = count
+        self.m = xqs[0].shape[0]
+        self.xq_arr = (C.c_void_p * count)(*[x.data_ptr() for x in xqs])
+        self.s_arr = (C.c_void_p * count)(*[s.data_ptr() for s in scales])
+        self.y_arr = (C.c_void_p * count)(*[y.data_ptr() for y in ys])
+        self.tw_arr = (TW * count)(*tws)
+        self.acc_arr = None
+        if accs is not None:
+            self.acc_arr = (C.c_void_p * count)(*[(a.data_ptr() if a is not None else None) for a in accs])
+        self._keep = (xqs, scales, ys, accs)
+
+    def __call__(self, flags=None, stream=None) -> None:
+        _check(load().bitnet_linear_q_grouped(self.xq_arr, self.s_arr, self.m, self.tw_arr, self.count,
+                                              self.y_arr, self.acc_arr, _ptr(flags), _stream(stream)),
+               "bitnet_linear_q_grouped")
+
+
+def linear_q_grouped(xqs, scales, tws, ys, accs=None, flags=None, stream=None) -> None:
+    GroupedCall(xqs, scales, tws, ys, accs)(flags=flags, stream=stream)
 
 
 class StackCall:

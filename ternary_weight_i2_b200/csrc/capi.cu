@@ -24,6 +24,9 @@ bool gemm_available();
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
                         int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace,
                         cudaStream_t st);
+cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
+                                int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace, cudaStream_t st);
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -655,6 +658,35 @@ bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t 
     }
     cudaError_t e = launch_gemm(xq, act_scale, m, w, y, acc_out, d_flags, wait_limit(), dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
+}
+
+bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                      const bitnet_tw *w, int64_t count, float *const *y, int32_t *const *acc_out,
+                                      int32_t *d_flags, void *stream)
+{
+    if (!xq || !act_scale || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: NULL array");
+    if (count < 1 || count > BITNET_GROUP_MAX)
+        return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: count=%lld out of range [1, %d]", (long long)count,
+                    BITNET_GROUP_MAX);
+    if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: bad m");
+    for (int64_t i = 0; i < count; ++i) {
+        bitnet_status s = check_tw(w[i], i);
+        if (s != BITNET_OK) return s;
+        if (!xq[i] || !act_scale[i] || !y[i])
+            return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: layer %lld has a NULL pointer", (long long)i);
+        if (!aligned(xq[i], 16) || !aligned(y[i], 16))
+            return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: layer %lld xq or y not 16-byte aligned",
+                        (long long)i);
+    }
+    DevInfo dev;
+    bitnet_status s = check_device(&dev);
+    if (s != BITNET_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m <= BITNET_GEMV_MAX_M)
+        return gemv_slices(nullptr, xq, act_scale, m, w, count, y, acc_out, d_flags, st, dev);
+    cudaError_t e = launch_gemm_grouped(xq, act_scale, m, w, int(count), y, acc_out, d_flags, wait_limit(),
+                                        dev.sm_count, g_trace, st);
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "grouped gemm launch");
 }
 
 bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet_tw *w, int64_t count,

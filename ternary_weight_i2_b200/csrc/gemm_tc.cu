@@ -34,6 +34,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 
 namespace bitnet {
@@ -53,22 +56,48 @@ constexpr int kEpiWarp0 = 7, kEpiThreads = 128;
 constexpr int kTmemCols = 2 * kBN;                 // two int32 accumulators
 constexpr int kGemmSmem = 1024 + kOOff + 4 * 2 * kStageOut;
 
-struct GemmParams {
+struct GemmProblem {
     CUtensorMap tmap_a;       // int8 q [M, Kpad]: dims {Kpad, M}, box {128, 128}, 128-byte swizzle
     CUtensorMap tmap_b;       // packed [N, 32*KB]: dims {32*KB, N}, box {32, 256}, no swizzle
     CUtensorMap tmap_y;       // fp32 y [M, N]: dims {N, M}, box {32, 32}, 128-byte swizzle (when tma_out)
     CUtensorMap tmap_acc;     // int32 acc [M, N], same shape (when tma_out and acc)
-    int32_t tma_out;          // outputs through TMA stores (N % 4 == 0), else direct stores
     const float *act_scale;   // [M]
     float *y;                 // [M, N]
     int32_t *acc;             // [M, N] or null
     float w_scale;
     int32_t m, n, kb;
     int32_t tiles_m, tiles_n;
+    int32_t tma_out;          // outputs through TMA stores (N % 4 == 0), else direct stores
+    int32_t tile0;            // first id of this problem's tiles in the launch's tile numbering
+};
+
+constexpr int kMaxGroup = 8;         // problems (layers) per launch
+constexpr int kMaxGemmCtas = 160;
+constexpr int kMaxGemmTiles = 3072;  // tiles per launch
+
+struct GemmParams {
+    GemmProblem prob[kMaxGroup];
+    int32_t nprob;
+    int32_t ntiles_total;
     int32_t *flags;
     uint64_t wait_limit;
     uint64_t *trace;          // optional: CTA 0 per-K-block globaltimer stamps (kGemmTraceBlocks x 8)
+    int32_t cta_off[kMaxGemmCtas + 1];   // CTA c runs tiles[cta_off[c] .. cta_off[c+1])
+    int32_t tiles[kMaxGemmTiles];        // tile ids, heaviest first within each CTA
 };
+static_assert(sizeof(GemmParams) <= 32760, "GEMM parameter block too large");
+
+struct TileRef {
+    int g, m_tile, n_tile;
+};
+
+__device__ __forceinline__ TileRef decode_tile(const GemmParams &p, int id)
+{
+    int g = 0;
+    while (g + 1 < p.nprob && id >= p.prob[g + 1].tile0) ++g;
+    const int local = id - p.prob[g].tile0;
+    return TileRef{g, local % p.prob[g].tiles_m, local / p.prob[g].tiles_m};
+}
 
 // Trace of CTA 0 (profiling aid), per K block it < kGemmTraceBlocks:
 // [it*8 + 0] producer issued, 1 MMA saw full, 2 MMA saw B ready, 3 MMA issued,
@@ -175,8 +204,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint64_t limit = p.wait_limit;
-    const int ntiles = p.tiles_m * p.tiles_n;
-    const int kblocks = p.kb;
+    const int tbeg = p.cta_off[blockIdx.x], tend = p.cta_off[blockIdx.x + 1];
     const uint32_t sbase = smem_u32(smem);
     uint64_t *ctrace = (p.trace && blockIdx.x == 0) ? p.trace + kGemmTraceBlocks * 8 : nullptr;
     if (ctrace && tid == 0) ctrace[0] = globaltimer();
@@ -225,8 +253,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
             const uint64_t pol_w = l2_evict_first_policy();
             int it = 0, last = -1;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const int m_tile = t % p.tiles_m, n_tile = t / p.tiles_m;
+            for (int ti = tbeg; ti < tend && ok; ++ti) {
+                const TileRef tr = decode_tile(p, p.tiles[ti]);
+                const GemmProblem &P = p.prob[tr.g];
+                const int m_tile = tr.m_tile, n_tile = tr.n_tile, kblocks = P.kb;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int s = it % kStages, r = it / kStages;
                     if (r > 0 && !wait_or_abort(smem_u32(&empty_bar[s]), (r - 1) & 1, limit, abort_flag)) {
@@ -239,9 +269,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                     asm volatile(
                         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
                         " [%0], [%1, {%2, %3}], [%4];" ::"r"(sbase + kAOff + s * kAStage),
-                        "l"(&p.tmap_a), "r"(kb * kBK), "r"(m_tile * kBM), "r"(fb)
+                        "l"(&P.tmap_a), "r"(kb * kBK), "r"(m_tile * kBM), "r"(fb)
                         : "memory");
-                    tma_load_2d(sbase + kPOff + s * kPStage, &p.tmap_b, kb * 32, n_tile * kBN, fb, pol_w);
+                    tma_load_2d(sbase + kPOff + s * kPStage, &P.tmap_b, kb * 32, n_tile * kBN, fb, pol_w);
                     stamp(it, 0);
                     last = it;
                 }
@@ -255,7 +285,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
         if (lane == 0) {
             int it = 0, tcount = 0;
             bool ok = true, any = false;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+            for (int ti = tbeg; ti < tend && ok; ++ti, ++tcount) {
+                const int kblocks = p.prob[decode_tile(p, p.tiles[ti]).g].kb;
                 const int b = tcount & 1, ur = tcount >> 1;
                 if (ur > 0 && !wait_or_abort(smem_u32(&acce_bar[b]), (ur - 1) & 1, limit, abort_flag)) {
                     fail();
@@ -301,7 +332,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
         const int c = lane & 7, rg = lane >> 3;
         int it = 0, tcount = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+        for (int ti = tbeg; ti < tend && ok; ++ti, ++tcount) {
+            const int kblocks = p.prob[decode_tile(p, p.tiles[ti]).g].kb;
             const int b = tcount & 1, ur = tcount >> 1;
             int32_t ps[kBM / 4];
 #pragma unroll
@@ -355,7 +387,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
         const int et = tid - 32 * kExpandWarp0;
         int it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int ti = tbeg; ti < tend && ok; ++ti) {
+            const int kblocks = p.prob[decode_tile(p, p.tiles[ti]).g].kb;
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 const int s = it % kStages, r = it / kStages;
                 const int bb = it % kBBufs, rb = it / kBBufs;
@@ -399,8 +432,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
         const int sub = warp & 3;            // TMEM lanes 32*sub .. 32*sub+31
         const uint32_t stage0 = sbase + kOOff + uint32_t(sub) * 2 * kStageOut;
         int tcount = 0, chunk_no = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
-            const int m_tile = t % p.tiles_m, n_tile = t / p.tiles_m;
+        for (int ti = tbeg; ti < tend; ++ti, ++tcount) {
+            const TileRef tr = decode_tile(p, p.tiles[ti]);
+            const GemmProblem &P = p.prob[tr.g];
+            const int m_tile = tr.m_tile, n_tile = tr.n_tile;
             const int b = tcount & 1, ur = tcount >> 1;
             const bool ready = wait_or_abort(smem_u32(&accf_bar[b]), ur & 1, limit, abort_flag);
             if (!__all_sync(0xffffffffu, ready)) {
@@ -410,8 +445,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
             tc_fence_after();
             const int rloc = 32 * sub + lane;
             const int row = m_tile * kBM + rloc;
-            const bool row_ok = row < p.m;
-            const float sa = row_ok ? p.act_scale[row] : 0.f;
+            const bool row_ok = row < P.m;
+            const float sa = row_ok ? P.act_scale[row] : 0.f;
             const int32_t rs = rowsum[b][rloc];
             const uint32_t taddr = tmem_base + (uint32_t(32 * sub) << 16) + uint32_t(b * kBN);
 #pragma unroll 1
@@ -419,8 +454,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                 uint32_t v[32];
                 tmem_ld32(taddr + uint32_t(c0), v);
                 const int col0 = n_tile * kBN + c0;
-                if (col0 >= p.n) continue;
-                if (p.tma_out) {
+                if (col0 >= P.n) continue;
+                if (P.tma_out) {
                     // stage the 32 x 32 chunk (row = lane) in the 128-byte swizzled
                     // layout and store it with one TMA store; tails are clipped by
                     // the tensor map
@@ -433,20 +468,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                         const int32_t a2 = int32_t(v[4 * j + 2]) - rs, a3 = int32_t(v[4 * j + 3]) - rs;
                         const uint32_t dst = stg + uint32_t(lane) * 128 + (uint32_t(j ^ (lane & 7)) << 4);
                         asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                                     "f"(__fmul_rn(__fmul_rn(float(a0), sa), p.w_scale)),
-                                     "f"(__fmul_rn(__fmul_rn(float(a1), sa), p.w_scale)),
-                                     "f"(__fmul_rn(__fmul_rn(float(a2), sa), p.w_scale)),
-                                     "f"(__fmul_rn(__fmul_rn(float(a3), sa), p.w_scale))
+                                     "f"(__fmul_rn(__fmul_rn(float(a0), sa), P.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a1), sa), P.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a2), sa), P.w_scale)),
+                                     "f"(__fmul_rn(__fmul_rn(float(a3), sa), P.w_scale))
                                      : "memory");
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&p.tmap_y, stg, col0, m_tile * kBM + 32 * sub);
+                        tma_store_2d(&P.tmap_y, stg, col0, m_tile * kBM + 32 * sub);
                         bulk_commit();
                     }
                     ++chunk_no;
-                    if (p.acc) {
+                    if (P.acc) {
                         const uint32_t stg2 = stage0 + uint32_t(chunk_no & 1) * kStageOut;
                         if (lane == 0) bulk_wait_read<1>();
                         __syncwarp();
@@ -461,20 +496,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(&p.tmap_acc, stg2, col0, m_tile * kBM + 32 * sub);
+                            tma_store_2d(&P.tmap_acc, stg2, col0, m_tile * kBM + 32 * sub);
                             bulk_commit();
                         }
                         ++chunk_no;
                     }
                 } else {
                     if (!row_ok) continue;
-                    float *yr = p.y + size_t(row) * size_t(p.n) + col0;
-                    int32_t *ar = p.acc ? p.acc + size_t(row) * size_t(p.n) + col0 : nullptr;
+                    float *yr = P.y + size_t(row) * size_t(P.n) + col0;
+                    int32_t *ar = P.acc ? P.acc + size_t(row) * size_t(P.n) + col0 : nullptr;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        if (col0 + j < p.n) {
+                        if (col0 + j < P.n) {
                             const int32_t a = int32_t(v[j]) - rs;
-                            yr[j] = __fmul_rn(__fmul_rn(float(a), sa), p.w_scale);
+                            yr[j] = __fmul_rn(__fmul_rn(float(a), sa), P.w_scale);
                             if (ar) ar[j] = a;
                         }
                     }
@@ -513,71 +548,127 @@ static PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn()
 
 bool gemm_available() { return true; }
 
-cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace,
-                        cudaStream_t st)
+// One or more grouped launches over `count` (<= kMaxGroup) problems sharing
+// the token count m.  Tiles are dealt heaviest-first to the least-loaded CTA
+// (cost = K blocks + a fixed epilogue share), so layers of different K
+// balance inside one persistent launch.
+cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
+                                int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace, cudaStream_t st)
 {
+    if (count < 1 || count > kMaxGroup) return cudaErrorInvalidValue;
     auto enc = gemm_encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    static thread_local GemmParams p;   // staging; copied into the launch
-    const int64_t kb = (w->k + 127) / 128;
-    {
-        const cuuint64_t dims[2] = {cuuint64_t(128 * kb), cuuint64_t(m)};
-        const cuuint64_t strides[1] = {cuuint64_t(128 * kb)};
-        const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kBM)};
+    static thread_local GemmParams p;   // staging; copied into each launch
+    struct Tile {
+        int id, cost;
+    };
+    static thread_local std::vector<Tile> all;
+    all.clear();
+    int tile0 = 0;
+    for (int g = 0; g < count; ++g) {
+        GemmProblem &P = p.prob[g];
+        const int64_t kb = (w[g].k + 127) / 128;
         const cuuint32_t es[2] = {1u, 1u};
-        if (enc(&p.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(xq), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+        {
+            const cuuint64_t dims[2] = {cuuint64_t(128 * kb), cuuint64_t(m)};
+            const cuuint64_t strides[1] = {cuuint64_t(128 * kb)};
+            const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kBM)};
+            if (enc(&P.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(xq[g]), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        {
+            const cuuint64_t dims[2] = {cuuint64_t(32 * kb), cuuint64_t(w[g].n)};
+            const cuuint64_t strides[1] = {cuuint64_t(32 * kb)};
+            const cuuint32_t box[2] = {32u, uint32_t(kBN)};
+            if (enc(&P.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w[g].packed), dims, strides, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        P.tma_out = (w[g].n % 4 == 0) ? 1 : 0;
+        int32_t *accg = acc ? acc[g] : nullptr;
+        if (P.tma_out) {
+            const cuuint64_t dims[2] = {cuuint64_t(w[g].n), cuuint64_t(m)};
+            const cuuint64_t strides[1] = {cuuint64_t(w[g].n) * 4};
+            const cuuint32_t box[2] = {32u, 32u};
+            if (enc(&P.tmap_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y[g], dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+            if (accg && enc(&P.tmap_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, accg, dims, strides, box, es,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        P.act_scale = act_scale[g];
+        P.y = y[g];
+        P.acc = accg;
+        P.w_scale = w[g].scale;
+        P.m = int32_t(m);
+        P.n = int32_t(w[g].n);
+        P.kb = int32_t(kb);
+        P.tiles_m = int32_t((m + kBM - 1) / kBM);
+        P.tiles_n = int32_t((w[g].n + kBN - 1) / kBN);
+        P.tile0 = tile0;
+        const int nt = P.tiles_m * P.tiles_n;
+        for (int i = 0; i < nt; ++i) all.push_back(Tile{tile0 + i, int(kb) + 3});
+        tile0 += nt;
     }
-    {
-        const cuuint64_t dims[2] = {cuuint64_t(32 * kb), cuuint64_t(w->n)};
-        const cuuint64_t strides[1] = {cuuint64_t(32 * kb)};
-        const cuuint32_t box[2] = {32u, uint32_t(kBN)};
-        const cuuint32_t es[2] = {1u, 1u};
-        if (enc(&p.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(w->packed), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    p.tma_out = (w->n % 4 == 0) ? 1 : 0;
-    if (p.tma_out) {
-        const cuuint64_t dims[2] = {cuuint64_t(w->n), cuuint64_t(m)};
-        const cuuint64_t strides[1] = {cuuint64_t(w->n) * 4};
-        const cuuint32_t box[2] = {32u, 32u};
-        const cuuint32_t es[2] = {1u, 1u};
-        if (enc(&p.tmap_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-        if (acc && enc(&p.tmap_acc, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, acc, dims, strides, box, es,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    p.act_scale = act_scale;
-    p.y = y;
-    p.acc = acc;
-    p.w_scale = w->scale;
-    p.m = int32_t(m);
-    p.n = int32_t(w->n);
-    p.kb = int32_t(kb);
-    p.tiles_m = int32_t((m + kBM - 1) / kBM);
-    p.tiles_n = int32_t((w->n + kBN - 1) / kBN);
+    p.nprob = count;
+    p.ntiles_total = tile0;
     p.flags = flags;
     p.wait_limit = wait_limit;
     p.trace = trace;
+    std::stable_sort(all.begin(), all.end(), [](const Tile &a, const Tile &b) { return a.cost > b.cost; });
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(gemm_i2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const int64_t tiles = int64_t(p.tiles_m) * p.tiles_n;
-    const int grid = int(tiles < sm_count ? tiles : sm_count);
-    gemm_i2_kernel<<<grid, kGemmThreads, kGemmSmem, st>>>(p);
-    return cudaGetLastError();
+    static thread_local std::vector<int> owner, fill;
+    for (size_t c0 = 0; c0 < all.size(); c0 += kMaxGemmTiles) {
+        const int n = int(std::min<size_t>(kMaxGemmTiles, all.size() - c0));
+        const int G = std::min(std::min(sm_count, kMaxGemmCtas), n);
+        // least-loaded CTA first (loads are small integers: linear scan)
+        static thread_local std::vector<long long> load;
+        load.assign(G, 0);
+        owner.assign(n, 0);
+        std::vector<int> count_of(G, 0);
+        for (int i = 0; i < n; ++i) {
+            int best = 0;
+            for (int c = 1; c < G; ++c)
+                if (load[c] < load[best]) best = c;
+            load[best] += all[c0 + i].cost;
+            owner[i] = best;
+            ++count_of[best];
+        }
+        p.cta_off[0] = 0;
+        for (int c = 0; c < G; ++c) p.cta_off[c + 1] = p.cta_off[c] + count_of[c];
+        fill.assign(G, 0);
+        for (int i = 0; i < n; ++i) {
+            const int c = owner[i];
+            p.tiles[p.cta_off[c] + fill[c]++] = all[c0 + i].id;
+        }
+        gemm_i2_kernel<<<G, kGemmThreads, kGemmSmem, st>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
+                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace,
+                        cudaStream_t st)
+{
+    const int8_t *xqa[1] = {xq};
+    const float *sa[1] = {act_scale};
+    float *ya[1] = {y};
+    int32_t *aa[1] = {acc};
+    return launch_gemm_grouped(xqa, sa, m, w, 1, ya, acc ? aa : nullptr, flags, wait_limit, sm_count, trace, st);
 }
 
 }  // namespace bitnet

@@ -93,3 +93,72 @@ def test_prefill_2048_sampled(shape):
     # |acc| is bounded by sum_k |q| for ternary weights
     q, _, _ = oracle.quant_act(x)
     assert (np.abs(ag.astype(np.int64)) <= np.abs(q.astype(np.int64)).sum(axis=1)[:, None]).all()
+
+
+def _grouped(xs, ws, scales, shared_index=None):
+    """Run bitnet_linear_q_grouped over layers (x_i, w_i); returns y, acc lists."""
+    xq_dev, s_dev = {}, {}
+    keys = shared_index or list(range(len(ws)))
+    for key, x in zip(keys, xs):
+        if key not in xq_dev:
+            q, s, _ = oracle.quant_act(x)
+            xq_dev[key], s_dev[key] = upload(q), upload(s)
+    tws, ys, accs = [], [], []
+    for w, sw in zip(ws, scales):
+        n, k = w.shape
+        pk = pack_on_gpu(w)
+        tws.append(tw2.make_tw(pk, n, k, sw))
+        ys.append(Guarded((xs[0].shape[0], n), torch.float32))
+        accs.append(Guarded((xs[0].shape[0], n), torch.int32))
+        tws[-1]._keep = pk
+    fl = flags_tensor()
+    tw2.linear_q_grouped([xq_dev[k] for k in keys], [s_dev[k] for k in keys], tws, [y.t for y in ys],
+                         [a.t for a in accs], flags=fl)
+    torch.cuda.synchronize()
+    assert int(fl.item()) == 0
+    for y, a in zip(ys, accs):
+        assert y.guard_intact() and a.guard_intact()
+    return [y.t.cpu().numpy() for y in ys], [a.t.cpu().numpy() for a in accs]
+
+
+def test_grouped_full_parity_mixed_shapes():
+    rng = np.random.default_rng(31)
+    m = 200
+    shapes = [(300, 1536), (256, 9024), (512, 1536), (100, 128)]
+    xa = synth.normal_row_spread(rng, m, 1536)
+    xb = synth.normal_row_spread(rng, m, 9024)
+    xc = synth.normal_row_spread(rng, m, 128)
+    xs = [xa, xb, xa, xc]
+    ws = [synth.ternary(rng, n, k) for n, k in shapes]
+    sc = [synth.weight_scale(rng) for _ in shapes]
+    ys, accs = _grouped(xs, ws, sc, shared_index=[0, 1, 0, 2])
+    for x, w, s, y, a in zip(xs, ws, sc, ys, accs):
+        pk_np, _ = oracle.pack(w)
+        a_want, y64, y32, _ = oracle.linear(x, pk_np, w.shape[0], w.shape[1], s)
+        np.testing.assert_array_equal(a, a_want)
+        np.testing.assert_array_equal(y.view(np.uint32), y32.view(np.uint32))
+        assert rel_err(y, y64) <= RTOL
+
+
+def test_grouped_prefill_2048_seven_shapes_sampled():
+    """The launch bench.py times: all seven decoder shapes at M = 2048 in one call."""
+    xs_by_k = synth.prefill_inputs(2048)
+    xs, ws, sc, keys = [], [], [], []
+    for i, (name, n, k) in enumerate(synth.LAYER_SHAPES):
+        rng = np.random.default_rng(synth.seed_for(4, i))
+        ws.append(synth.ternary(rng, n, k))
+        sc.append(synth.weight_scale(rng))
+        xs.append(xs_by_k[k])
+        keys.append(k)
+    ys, accs = _grouped(xs, ws, sc, shared_index=keys)
+    rng = np.random.default_rng(5)
+    for x, w, s, y, a in zip(xs, ws, sc, ys, accs):
+        n, k = w.shape
+        cols = np.unique(np.concatenate([[0, n - 1], rng.choice(n, 6, replace=False)]))
+        pk_np, _ = oracle.pack(w[cols])
+        a_want, _, y32, _ = oracle.linear(x, pk_np, len(cols), k, s)
+        np.testing.assert_array_equal(a[:, cols], a_want)
+        np.testing.assert_array_equal(y[:, cols].view(np.uint32), y32.view(np.uint32))
+        _, s_act, _ = oracle.quant_act(x)
+        y_all = (a.astype(np.float32) * s_act[:, None]).astype(np.float32) * np.float32(s)
+        np.testing.assert_array_equal(y.view(np.uint32), y_all.view(np.uint32))
