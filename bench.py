@@ -425,7 +425,7 @@ def run_prefill(dev, stream, flags, world):
                          "unit": "TOPS", "frac": round(tops / world / peak, 4),
                          "peak_kind": "measured bf16 cuBLAS burst (MEASURED_PEAKS.json) x 2 (int8:bf16 dense ratio)"},
             "quant_ms_per_step": round(tq, 5), "per_shape": per_shape,
-            "kernel": "gemm_i2_kernel (tcgen05.mma kind::i8, 128x256x128 tiles, one grouped launch)"}
+            "kernel": "gemm_i2_kernel (tcgen05.mma kind::i8, weights expanded into TMEM as A, activations as B from shared memory, 128 features x 192 tokens x 128 tiles, one grouped launch)"}
 
 
 def build_stack_views(m, dev, tws, layers=28):

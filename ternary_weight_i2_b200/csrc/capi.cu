@@ -22,11 +22,12 @@ cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float
                          cudaStream_t st);
 bool gemm_available();
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace,
-                        cudaStream_t st);
+                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count,
+                        uint64_t *trace, cudaStream_t st);
 cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
                                 const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
-                                int32_t *flags, uint64_t wait_limit, int sm_count, uint64_t *trace, cudaStream_t st);
+                                int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count, uint64_t *trace,
+                                cudaStream_t st);
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -633,7 +634,7 @@ bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_tw *w, float
     float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + qa);
     cudaError_t e = launch_quant(x, m, w->k, xq, xs, d_flags, st);
     if (e != cudaSuccess) return cuda_fail(e, "quant launch");
-    e = launch_gemm(xq, xs, m, w, y, acc_out, d_flags, wait_limit(), dev.sm_count, g_trace, st);
+    e = launch_gemm(xq, xs, m, w, y, acc_out, d_flags, wait_limit(), g_force_stall, dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 
@@ -656,7 +657,7 @@ bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t 
         int32_t *aa[1] = {acc_out};
         return gemv_slices(nullptr, xqa, xsa, m, w, 1, ya, aa, d_flags, st, dev);
     }
-    cudaError_t e = launch_gemm(xq, act_scale, m, w, y, acc_out, d_flags, wait_limit(), dev.sm_count, g_trace, st);
+    cudaError_t e = launch_gemm(xq, act_scale, m, w, y, acc_out, d_flags, wait_limit(), g_force_stall, dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 
@@ -685,7 +686,7 @@ bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *cons
     if (m <= BITNET_GEMV_MAX_M)
         return gemv_slices(nullptr, xq, act_scale, m, w, count, y, acc_out, d_flags, st, dev);
     cudaError_t e = launch_gemm_grouped(xq, act_scale, m, w, int(count), y, acc_out, d_flags, wait_limit(),
-                                        dev.sm_count, g_trace, st);
+                                        g_force_stall, dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "grouped gemm launch");
 }
 

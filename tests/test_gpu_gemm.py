@@ -162,3 +162,37 @@ def test_grouped_prefill_2048_seven_shapes_sampled():
         _, s_act, _ = oracle.quant_act(x)
         y_all = (a.astype(np.float32) * s_act[:, None]).astype(np.float32) * np.float32(s)
         np.testing.assert_array_equal(y.view(np.uint32), y_all.view(np.uint32))
+
+
+def test_gemm_forced_timeout_returns_status_and_context_survives():
+    """The prefill kernel's bounded waits: with the test aid on, one K block's
+    copies are never issued; the expanders' wait for them runs out, the launch
+    ends with the timeout flag (every role still passes its barriers), and the
+    next call is correct."""
+    rng = np.random.default_rng(17)
+    m, k, n = 200, 1536, 1536
+    w = synth.ternary(rng, n, k)
+    x = synth.normal_row_spread(rng, m, k)
+    s_w = synth.weight_scale(rng)
+    pk = pack_on_gpu(w)
+    tw = tw2.make_tw(pk, n, k, s_w)
+    y = torch.zeros((m, n), dtype=torch.float32, device=DEV)
+    ws = torch.empty(tw2.linear_workspace_bytes(m, k), dtype=torch.uint8, device=DEV)
+    fl = flags_tensor()
+    try:
+        tw2._abi.set_wait_limit(20000)
+        tw2._abi.force_stall(True)
+        tw2.linear(upload(x), tw, y, workspace=ws, flags=fl)
+        torch.cuda.synchronize()
+    finally:
+        tw2._abi.force_stall(False)
+        tw2._abi.set_wait_limit(0)
+    assert int(fl.item()) & tw2.FLAG_TIMEOUT
+    assert tw2.status_from_flags(int(fl.item())) == tw2._abi.ERR_TIMEOUT
+    fl.zero_()
+    tw2.linear(upload(x), tw, y, workspace=ws, flags=fl)
+    torch.cuda.synchronize()
+    assert int(fl.item()) == 0
+    pk_np, _ = oracle.pack(w)
+    _, _, y32, _ = oracle.linear(x, pk_np, n, k, s_w)
+    np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), y32.view(np.uint32))
