@@ -273,16 +273,14 @@ BITNET_API bitnet_status bitnet_debug_force_stall(int on);
  * 1 first weight copies issued, 2 activations quantised, 3 first chunk landed,
  * 4 last chunk consumed (other slots unused).  The buffer must hold
  * 8 * warps * CTAs entries (at most 8 * 16 * 160).  Tensor-core GEMM launches
- * (m > 8) write SM clock (clock64) stamps of the first SM pair, CTA r at
- * d_trace[1024*r + ...] (2048 entries in all): for its first 48 K blocks it,
- * [it*16 + e]: e = 0 TMA issued, 1 the pair's second half of A written (first
- * CTA), 2/3 MMA warp passed its barrier / issued the MMAs, 4+q / 8+q / 12+q
- * expander warp of TMEM lane quadrant q saw the tile / a free weight buffer /
- * finished writing it; then [768 + 0] kernel entry, [768 + 1] set-up done,
- * [768 + 2] all roles done, [768 + 3] / [768 + 4] %globaltimer (ns) at entry /
- * at the end, [768 + 8 + t] epilogue of tile t done, [768 + 24 + t] MMA warp
- * passed tile t's accumulator barrier (t < 16).  A stamp taken just after a
- * barrier instruction can precede the barrier's completion.
+ * (m > 8) write SM clock (clock64) stamps of CTA 0: for its first 48 K blocks
+ * it, d_trace[it*16 + e]: e = 0 TMA issued, 1/2 MMA thread saw the tile / the
+ * expanded weights, 3 MMAs issued, 4+q / 8+q / 12+q expander warp of TMEM lane
+ * quadrant q saw the tile / a free weight buffer / finished writing it; then
+ * d_trace[768 + 0] kernel entry, [768 + 1] set-up done, [768 + 2] all roles
+ * done, [768 + 3] / [768 + 4] %globaltimer (ns) at entry / at the end,
+ * [768 + 8 + t] epilogue of the CTA's tile t done and [768 + 24 + t] MMA
+ * thread found tile t's accumulator free (t < 16).
  * NULL turns it off. */
 BITNET_API bitnet_status bitnet_debug_set_trace(void *d_trace);
 

@@ -1,5 +1,5 @@
 // gemm_tc.cu -- prefill path (M > 8 tokens): ternary x int8 GEMM on the
-// 5th-generation tensor cores (tcgen05, kind::i8), two SMs per MMA.
+// 5th-generation tensor cores (tcgen05, kind::i8).
 //
 // What it computes ("VibeVoice-ASR-BitNet Technical Report", §2.2.2, §2.4.2,
 // Figure 4; prefill in §3.2, Figure 6a): for int8 activations q [M, Kpad]
@@ -14,38 +14,35 @@
 // Operand roles.  The weights are the MMA's A operand and live in tensor
 // memory (TMEM); the activations are B and come from shared memory, so the
 // accumulator is D[n, m] = sum_k w[n,k] q[m,k]: one TMEM lane per output
-// feature, one column per token.  Expanded weights never touch shared memory.
+// feature, one column per token.  The expanded weights never touch shared
+// memory: per K block shared memory carries only the TMA-landed activation
+// and packed-weight tiles and the tensor core's read of the activations
+// (shared-memory bandwidth, not the tensor pipe, bounds a design that stages
+// expanded weights there).
 //
-// Two SMs per MMA.  A cluster of two CTAs computes tiles of 256 features x up
-// to 192 tokens with tcgen05.mma.cta_group::2 (M = 256): each CTA holds 128
-// weight rows in its own TMEM and half of the tile's tokens in its own
-// shared memory, and its TMEM receives its 128 rows of D.  Per K block an SM
-// thus loads 96 activation rows + 128 packed weight rows (16 KB) for the
-// work of 128 x 192 x 128 MACs: half the activation traffic of one SM doing
-// the same tile alone, and room for a 12-stage copy ring.
-//
-// Roles per CTA (16 warps), per 128-element K block:
-//   warps 0, 3     TMA producers: this CTA's 96 x 128 B activation half
-//                  (128-byte swizzle, the canonical K-major layout of B) and
-//                  its 128 x 32 B packed weight rows, into a 12-stage ring;
-//   warps 4-11     expanders, one thread per weight row: the row's 32 packed
-//                  bytes become 128 signed int8 weights (logic ops and one
-//                  add per 4 weights) written to one of 4 TMEM A buffers with
-//                  one tcgen05.st; two groups of four warps take alternate K
-//                  blocks;
-//   warps 12-15    epilogue: tcgen05.ld 32 tokens of a feature per thread,
-//                  dequantise in fp32, store (a warp writes 32 consecutive
-//                  features of one token per store);
-//   warp 1         (first CTA of the pair) issues the four tcgen05.mma of each
-//                  K block for both SMs and commits to the barriers of both
-//                  CTAs at once (multicast commit);
-//   warp 2         (first CTA) relay: turns the second CTA's remote mbarrier
-//                  signals into named-barrier arrivals for the MMA warp.
-// The MMA warp waits only on hardware named barriers (an mbarrier poll in
-// the issuing warp idles the tensor core for over a hundred cycles per K
-// block); every other wait is bounded, and every role arrives exactly once
-// per barrier phase, also after a timeout, so the MMA warp always completes.
-// No TMA multicast: each CTA loads only into its own shared memory.
+// One CTA per SM, persistent over tiles of 128 features x up to 192 tokens;
+// per 128-element K block (one packed block per weight row):
+//   warps 0, 2, 3  TMA: the activation tile (192 tokens x 128 B, 128-byte
+//                  swizzle: the canonical K-major layout of B) and the packed
+//                  weight tile (128 rows x 32 B) into a 7-stage ring; K block
+//                  `it` is issued by producer it % 3;
+//   warps 4-11     expanders, one thread per weight row: read the row's 32
+//                  packed bytes, turn the 2-bit codes into signed int8 w in
+//                  registers (three logic ops and one add per 4 weights, no
+//                  multiply) and write the row's 128 values, 32 TMEM columns,
+//                  with one tcgen05.st into one of 4 A buffers; two groups of
+//                  four warps take alternate K blocks;
+//   warp 1         one thread issues 4 tcgen05.mma (M=128, N<=192, K=32, A
+//                  from TMEM, B from shared memory, both signed) per K block
+//                  into one of two TMEM accumulators, so the epilogue of one
+//                  tile overlaps the next tile's K loop, and commits to
+//                  mbarriers;
+//   warps 12-15    epilogue: tcgen05.ld gives each thread 32 tokens of one
+//                  feature; dequantise in fp32 and store, each warp writing 32
+//                  consecutive features (128 bytes) of one token per store.
+// Every wait is bounded; on expiry the CTA raises BITNET_FLAG_TIMEOUT, the
+// other roles stop, in-flight copies and MMAs are drained (bounded) and TMEM
+// is freed before exit.  No TMA multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -56,30 +53,27 @@
 
 namespace bitnet {
 
-constexpr int kBF = 128;                           // weight rows per CTA (TMEM lanes); 256 per pair
-constexpr int kPairF = 2 * kBF;                    // features per tile: MMA M
+constexpr int kBF = 128;                           // features per tile: MMA M, TMEM lanes
 constexpr int kBT = 192;                           // tokens per tile: MMA N (at most)
-constexpr int kHalfT = kBT / 2;                    // activation rows per CTA
 constexpr int kBK = 128;                           // K per block: one packed block per row
-constexpr int kStages = 12;                        // TMA ring (activation half + packed weights)
+constexpr int kStages = 7;                         // TMA ring (activations + packed weights)
 constexpr int kABufs = 4;                          // expanded weight tiles in TMEM
-constexpr int kActStage = kHalfT * kBK;            // 12 KB int8 activations
+constexpr int kActStage = kBT * kBK;               // 24 KB int8 activations
 constexpr int kPStage = kBF * 32;                  // 4 KB packed weights
 constexpr int kActOff = 0, kPOff = kStages * kActStage;
 constexpr int kGemmSmem = 1024 + kPOff + kStages * kPStage;
 constexpr int kGemmThreads = 512;                  // 16 warps
-constexpr int kProducers = 2;                      // TMA-issuing warps: 0, 3
+constexpr int kProducers = 3;                      // TMA-issuing warps: 0, 2, 3
 constexpr int kExpandWarp0 = 4, kExpandGroupWarps = 4, kExpandGroups = 2;
 constexpr int kEpiWarp0 = 12, kEpiWarps = 4;
 constexpr int kACol0 = 2 * kBT;                    // TMEM columns of the A buffers
 constexpr int kTmemCols = 512;
 static_assert(kACol0 + 32 * kABufs <= kTmemCols, "TMEM budget");
 static_assert(kGemmSmem <= 232448, "shared-memory budget");
-static_assert(kActStage % 1024 == 0, "128-byte-swizzled stages need 1024-byte alignment");
 static_assert(kEpiWarp0 % 4 == 0 && kExpandWarp0 % 4 == 0, "TMEM lane quadrant = warp % 4");
 
 struct GemmProblem {
-    CUtensorMap tmap_q;       // int8 q [M, Kpad]: dims {Kpad, M}, box {128, 96}, 128-byte swizzle
+    CUtensorMap tmap_q;       // int8 q [M, Kpad]: dims {Kpad, M}, box {128, 192}, 128-byte swizzle
     CUtensorMap tmap_w;       // packed [N, 32*KB]: dims {32*KB, N}, box {32, 128}, no swizzle
     const float *act_scale;   // [M]
     float *y;                 // [M, N]
@@ -91,7 +85,7 @@ struct GemmProblem {
 };
 
 constexpr int kMaxGroup = 8;         // problems (layers) per launch
-constexpr int kMaxGemmPairs = 80;
+constexpr int kMaxGemmCtas = 160;
 constexpr int kMaxGemmTiles = 7168;  // tiles per launch
 
 struct GemmParams {
@@ -101,9 +95,9 @@ struct GemmParams {
     int32_t *flags;
     uint64_t wait_limit;
     int32_t force_stall;      // test aid: K block kStallBlock's copies are never issued
-    uint64_t *trace;          // optional: the first pair's stamps (2 * kGemmTraceStride entries)
-    int32_t pair_off[kMaxGemmPairs + 1];   // pair c runs tiles[pair_off[c] .. pair_off[c+1])
-    int32_t tiles[kMaxGemmTiles];          // tile ids, heaviest first within each pair
+    uint64_t *trace;          // optional: CTA 0 stamps (kGemmTraceMisc + 72 entries)
+    int32_t cta_off[kMaxGemmCtas + 1];   // CTA c runs tiles[cta_off[c] .. cta_off[c+1])
+    int32_t tiles[kMaxGemmTiles];        // tile ids, heaviest first within each CTA
 };
 static_assert(sizeof(GemmParams) <= 32760, "GEMM parameter block too large");
 
@@ -119,19 +113,16 @@ __device__ __forceinline__ TileRef decode_tile(const GemmParams &p, int id)
     return TileRef{g, local / p.prob[g].tiles_t, local % p.prob[g].tiles_t};
 }
 
-// Trace of the first pair's two CTAs, CTA r at [r * kGemmTraceStride + ...]
-// (profiling aid; a stamp right after a named barrier may be taken before the
-// barrier has completed): SM clock stamps per K block it <
-// kGemmTraceBlocks at [it*16 + e]: 0 producer issued, 1 relay saw the second
-// CTA's A half written, 2 MMA warp passed the A barrier, 3 MMAs issued, 4+q / 8+q / 12+q expander warp of lane quadrant q
-// saw full / saw its A buffer free / wrote it; then at kGemmTraceMisc + 0
+// Trace of CTA 0 (profiling aid): SM clock stamps per K block it <
+// kGemmTraceBlocks at [it*16 + e]: 0 producer issued, 1 (a value, not a
+// stamp) 1 if the MMA thread's look-ahead found the block ready, else 2, 2 MMA
+// saw A ready, 3 MMA issued, 4+q / 8+q / 12+q expander warp of lane quadrant
+// q saw full / saw its A buffer free / wrote it; then at kGemmTraceMisc + 0
 // kernel entry, +1 set-up done, +2 all roles done, +3 / +4 globaltimer at
-// entry / end, +8+t epilogue of tile t done, +24+t MMA warp passed tile t's
-// accumulator barrier (t < 16), +40+16t+2c (+1) epilogue warp 0 loaded
-// (stored) chunk c of tile t (t < 2).
+// entry / end, +8+t epilogue of tile t done, +24+t MMA found tile t's
+// accumulator free (t < 16).
 constexpr int kGemmTraceBlocks = 48, kGemmTraceEv = 16;
 constexpr int kGemmTraceMisc = kGemmTraceBlocks * kGemmTraceEv;
-constexpr int kGemmTraceStride = 1024;             // entries per traced CTA (CTAs 0 and 1)
 
 // ------------------------------------------------------------ tcgen05 PTX
 
@@ -151,17 +142,16 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
 }
 
 // Instruction descriptor: kind::i8, D int32, A and B signed int8, both
-// K-major, M = 256 (two SMs), N = n (a multiple of 16, at most 256), dense.
+// K-major, M = 128, N = n (a multiple of 16, at most 256), dense.
 __device__ __forceinline__ uint32_t idesc_i8(int n)
 {
-    return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kPairF >> 4) << 24);
+    return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kBF >> 4) << 24);
 }
 
-// One K block for both SMs of the pair, issued by one thread of the first
-// CTA: four MMAs (K = 32 each) into d_tmem -- the activation descriptor of K
-// step ks is qdesc + 2*ks (32 bytes further, in 16-byte units; the
-// start-address field cannot carry out for shared-memory addresses) -- then
-// commits, to the barriers at the same offsets in both CTAs, that free the
+// One K block, issued by one thread: four MMAs (K = 32 each) into d_tmem --
+// the activation descriptor of K step ks is qdesc + 2*ks (32 bytes further,
+// in 16-byte units; the start-address field cannot carry out for
+// shared-memory addresses) -- then commits to the barriers that free the
 // activation stage and the A buffer.
 __device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_tmem, uint64_t qdesc, uint32_t idesc,
                                            uint32_t accumulate, uint32_t bar_stage, uint32_t bar_abuf)
@@ -170,41 +160,24 @@ __device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_tmem, uin
         "{\n\t.reg .pred p0, p1;\n\t"
         "setp.ne.b32 p0, %4, 0;\n\t"
         "setp.eq.u32 p1, %4, %4;\n\t"
-        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%6], %7, %3, p1;\n\t"
-        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%8], %9, %3, p1;\n\t"
-        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%10], %11, %3, p1;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%5], %13;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%12], %13;\n\t}"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%6], %7, %3, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%8], %9, %3, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%10], %11, %3, p1;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(qdesc), "r"(idesc), "r"(accumulate), "r"(bar_stage), "r"(a_tmem + 8u),
-          "l"(qdesc + 2u), "r"(a_tmem + 16u), "l"(qdesc + 4u), "r"(a_tmem + 24u), "l"(qdesc + 6u), "r"(bar_abuf),
-          "h"(uint16_t(3))
+          "l"(qdesc + 2u), "r"(a_tmem + 16u), "l"(qdesc + 4u), "r"(a_tmem + 24u), "l"(qdesc + 6u), "r"(bar_abuf)
         : "memory");
 }
 
-// Commit to the barrier at this offset in both CTAs of the pair.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-        "h"(uint16_t(3))
-        : "memory");
-}
-
-// Commit to this CTA's barrier only.
-__device__ __forceinline__ void mma_commit_local(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// Named (hardware) barriers of the first CTA between the MMA warp and the
-// warps that feed or drain TMEM: ids 1..4 "A buffer a written in both CTAs"
-// (the CTA's expander group of four warps + the relay warp + the MMA warp),
-// ids 5..6 "accumulator b drained in both CTAs" (four epilogue warps + relay
-// + MMA warp).  The MMA warp waits (bar.sync); the others arrive
-// (bar.arrive, release), exactly once per phase.
-constexpr uint32_t kNbAbuf0 = 1, kNbAcc0 = 5, kNbThreads = 192;
-static_assert(kNbThreads == 32 * (kExpandGroupWarps + 2) && kNbThreads == 32 * (kEpiWarps + 2), "barrier sizes");
+// Named (hardware) barriers between the MMA warp and the warps that feed or
+// drain the tensor memory: ids 1..4 "A buffer a written" (expander group of
+// four warps + the MMA warp), ids 5..6 "accumulator b drained" (four epilogue
+// warps + the MMA warp).  The MMA warp waits (bar.sync), the others arrive
+// (bar.arrive, release); each phase has exactly one arrival per warp.
+constexpr uint32_t kNbAbuf0 = 1, kNbAcc0 = 5, kNbThreads = 160;
+static_assert(kNbThreads == 32 * (kExpandGroupWarps + 1) && kNbThreads == 32 * (kEpiWarps + 1), "barrier sizes");
 __device__ __forceinline__ void nb_arrive(uint32_t id)
 {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kNbThreads) : "memory");
@@ -214,45 +187,13 @@ __device__ __forceinline__ void nb_sync(uint32_t id)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kNbThreads) : "memory");
 }
 
-__device__ __forceinline__ uint32_t cluster_rank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// All threads of both CTAs (release / acquire at cluster scope).
-__device__ __forceinline__ void cluster_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Arrive on the barrier at this offset in CTA `rank`.  Relaxed: what it
-// signals is the completion of this thread's TMEM accesses (tcgen05.wait::st
-// / wait::ld, then tcgen05.fence::before_thread_sync, precede it); a release
-// would also wait for every earlier global store of the thread (the
-// epilogue's outputs), which the MMA warp does not need.
-__device__ __forceinline__ void remote_arrive(uint32_t bar, uint32_t rank)
-{
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
-        "r"(rank)
-        : "memory");
-}
-
-// SM clock read ordered with the surrounding volatile asm (barriers, MMAs),
-// for the trace.
-__device__ __forceinline__ uint64_t clock_ordered()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t)::"memory");
-    return t;
-}
-
 // K block whose copies a test stalls (force_stall)
 constexpr int kStallBlock = 2;
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
 {
@@ -292,64 +233,51 @@ __device__ __forceinline__ uint32_t expand_signed(uint32_t v, int g)
     return (c - 0x01010101u) ^ 0x80808080u;
 }
 
-// Suspend-time hint of every wait: a waiting thread that polls without one
-// takes issue slots from the warps that work (the expanders above all), and
-// one suspended for long is not reliably woken at once by arrivals from the
-// other SM or from the asynchronous units -- a short hint bounds both.
-constexpr uint32_t kSleepNs = 100;
-
 // Wait on an mbarrier phase; false on timeout or when another role aborted.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uint64_t limit, volatile int *abort_flag)
+// Between polls the thread may sleep up to `sleep_ns` (it wakes as soon as
+// the phase completes), so roles that wait do not take issue slots from the
+// ones that work.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uint64_t limit, volatile int *abort_flag,
+                                              uint32_t sleep_ns = 0)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = clock64();
     for (int spin = 0;; ++spin) {
-        if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+        if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
         if ((spin & 15) == 0 && *abort_flag) return false;
         if (clock64() - t0 > limit) return false;
     }
 }
-
-// Cluster-scope acquire poll with the short suspend-time hint (the phases
-// it waits for may be completed by the other CTA's remote arrivals).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSleepNs)
-        : "memory");
-    return ok != 0;
-}
+// Suspend-time hint of the waiting roles: without one, a polling thread takes
+// issue slots from the warps that work; with a long one, a thread is not
+// reliably woken at once by arrivals of the asynchronous units (TMA, tensor
+// core commits) and the pipeline stalls -- a short hint bounds both.
+constexpr uint32_t kSleepNs = 100;
 
 // Warp-wide wait: lane 0 polls, the others take its result (and, through
-// __syncwarp, the ordering its successful wait established).
+// __syncwarp, the ordering its successful wait established).  One poller per
+// warp instead of 32 keeps the barrier traffic of the waiting roles low.
 __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity, uint64_t limit,
-                                                   volatile int *abort_flag)
+                                                   volatile int *abort_flag, uint32_t sleep_ns = kSleepNs)
 {
     bool ok = false;
-    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, limit, abort_flag);
+    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, limit, abort_flag, sleep_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     return ok;
 }
 
-// Warp-wide wait for a phase that is bound to complete: one the MMA warp's
-// commits complete (it never stops) -- `cluster` false -- or one the other
-// CTA's roles complete with remote arrivals (they arrive once per phase
-// whatever happens) -- `cluster` true, cluster-scope acquire.  No abort
-// check, only the long limit.
-__device__ __forceinline__ bool warp_wait_progress(uint32_t bar, uint32_t parity, uint64_t long_limit,
-                                                   bool cluster = false)
+// Warp-wide wait for a phase the MMA warp's commits complete: no abort
+// check (those commits always come), only the long limit.
+__device__ __forceinline__ bool warp_wait_progress(uint32_t bar, uint32_t parity, uint64_t long_limit)
 {
     bool ok = false;
     if ((threadIdx.x & 31) == 0) {
-        const uint64_t t0 = clock64();
-        while (!(ok = cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity, kSleepNs)) &&
-               clock64() - t0 <= long_limit) {
+        ok = mbar_try_wait(bar, parity);
+        if (!ok) {
+            const uint64_t t0 = clock64();
+            while (!(ok = mbar_try_wait_sleep(bar, parity, kSleepNs)) && clock64() - t0 <= long_limit) {
+            }
         }
     }
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -357,39 +285,33 @@ __device__ __forceinline__ bool warp_wait_progress(uint32_t bar, uint32_t parity
     return ok;
 }
 
-// Tokens of tile t_tile.
+// Tokens of tile t_tile and the MMA's N for them (a multiple of 16).
 __device__ __forceinline__ int tile_tokens(const GemmProblem &P, int t_tile)
 {
     return min(kBT, P.m - t_tile * kBT);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    gemm_i2_kernel(const __grid_constant__ GemmParams p)
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_constant__ GemmParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
     __shared__ __align__(8) uint64_t aempty_bar[kABufs], accf_bar[2], drain_bar;
-    __shared__ __align__(8) uint64_t peer_ready_bar[kABufs], peer_drained_bar[2];   // first CTA only
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     volatile int *abort_flag = &abort_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_rank();              // 0: issues the MMAs; 1: its peer
-    const bool leader = rank == 0;
     const uint64_t limit = p.wait_limit;
-    // limit of the waits that are bound to end (see warp_wait_progress): far
-    // above the time one failed copy wait can hold the pipeline up
+    // limit of the waits on the MMA warp's commits, which always come (the MMA
+    // warp never stops): far above the time one failed copy wait can hold
+    // the pipeline up
     const uint64_t long_limit = (limit > (kDrainWaitLimit >> 2)) ? (limit << 2) : kDrainWaitLimit;
-    const int pair = blockIdx.x >> 1;
-    const int tbeg = p.pair_off[pair], tend = p.pair_off[pair + 1];
+    const int tbeg = p.cta_off[blockIdx.x], tend = p.cta_off[blockIdx.x + 1];
     const uint32_t sbase = smem_u32(smem);
-    // trace: the first pair, each CTA in its own kGemmTraceStride block
-    uint64_t *const tbase = (p.trace && blockIdx.x < 2) ? p.trace + blockIdx.x * kGemmTraceStride : nullptr;
-    uint64_t *ctrace = tbase ? tbase + kGemmTraceMisc : nullptr;
+    uint64_t *ctrace = (p.trace && blockIdx.x == 0) ? p.trace + kGemmTraceMisc : nullptr;
     if (ctrace && tid == 0) {
-        ctrace[0] = clock_ordered();
+        ctrace[0] = clock64();
         ctrace[3] = globaltimer();
     }
 
@@ -398,60 +320,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             mbar_init(smem_u32(&full_bar[s]), 1);
             mbar_init(smem_u32(&empty_bar[s]), 1 + kExpandGroupWarps);   // MMA commit, expander warps
         }
-        for (int a = 0; a < kABufs; ++a) {
-            mbar_init(smem_u32(&aempty_bar[a]), 1);
-            mbar_init(smem_u32(&peer_ready_bar[a]), kExpandGroupWarps);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&accf_bar[b]), 1);
-            mbar_init(smem_u32(&peer_drained_bar[b]), kEpiWarps);
-        }
+        for (int a = 0; a < kABufs; ++a) mbar_init(smem_u32(&aempty_bar[a]), 1);
+        for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&accf_bar[b]), 1);
         mbar_init(smem_u32(&drain_bar), 1);
         abort_s = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
                      "r"(kTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // both CTAs' barriers are initialised (and TMEM allocated) before either
-    // CTA touches the other's
     tc_fence_before();
-    cluster_sync();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_s;
-    if (ctrace && tid == 0) ctrace[1] = clock_ordered();
+    if (ctrace && tid == 0) ctrace[1] = clock64();
 
     auto fail = [&]() {
         abort_s = 1;
         raise_flag(p.flags, BITNET_FLAG_TIMEOUT);
     };
-    uint64_t *trace = tbase;
+    uint64_t *trace = (p.trace && blockIdx.x == 0) ? p.trace : nullptr;
     auto stamp = [&](int it, int ev) {
-        if (trace && it < kGemmTraceBlocks) trace[it * kGemmTraceEv + ev] = clock_ordered();
+        if (trace && it < kGemmTraceBlocks) trace[it * kGemmTraceEv + ev] = clock64();
     };
 
-    if (warp == 0 || warp == 3) {
+    if (warp == 0 || warp == 2 || warp == 3) {
         // ----------------------------------------------------- TMA producers
         // The whole warp runs the loop and lane 0 issues the copies (a lone
         // diverged lane is starved by busy warps of its sub-partition).
-        const int pidx = (warp == 0) ? 0 : 1;
+        const int pidx = (warp == 0) ? 0 : warp - 1;
         int it = 0, last = -1;
         bool ok = true;
         for (int ti = tbeg; ti < tend && ok; ++ti) {
             const TileRef tr = decode_tile(p, p.tiles[ti]);
             const GemmProblem &P = p.prob[tr.g];
             const int kblocks = P.kb;
-            // this CTA's token half of the tile: the MMA's B rows [0, n/2) come
-            // from the first CTA, [n/2, n) from the second.  Box origins stay
-            // inside the tensors (a short last tile or a ragged feature count
-            // would otherwise start a box past the end); rows read in place of
-            // the missing ones only reach outputs that are never stored.
-            const int half = ((tile_tokens(P, tr.t_tile) + 15) & ~15) >> 1;
-            const int t_row = min(tr.t_tile * kBT + int(rank) * half, P.m - 1);
-            const int f_row = min(tr.f_tile * kPairF + int(rank) * kBF, P.n - 1);
             for (int kb = 0; kb < kblocks; ++kb, ++it) {
                 if (it % kProducers != pidx) continue;
                 const int s = it % kStages, r = it / kStages;
@@ -467,12 +373,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     asm volatile(
                         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
                         " [%0], [%1, {%2, %3}], [%4];" ::"r"(sbase + kActOff + s * kActStage),
-                        "l"(&P.tmap_q), "r"(kb * kBK), "r"(t_row), "r"(fb)
+                        "l"(&P.tmap_q), "r"(kb * kBK), "r"(tr.t_tile * kBT), "r"(fb)
                         : "memory");
                     asm volatile(
                         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
                         " [%0], [%1, {%2, %3}], [%4];" ::"r"(sbase + kPOff + s * kPStage),
-                        "l"(&P.tmap_w), "r"(kb * 32), "r"(f_row), "r"(fb)
+                        "l"(&P.tmap_w), "r"(kb * 32), "r"(tr.f_tile * kBF), "r"(fb)
                         : "memory");
                     stamp(it, 0);
                 }
@@ -487,97 +393,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
-        // First CTA only.  Waits only on named barriers, never gives up,
-        // always commits: every other role's waits on its commits therefore
-        // end.  The expanders (and, through the relay, the second CTA's)
+        // Waits only on the named barriers the expanders and the epilogue
+        // arrive at (an mbarrier poll here costs the tensor core more than a
+        // hundred cycles per K block), never gives up, always commits: every
+        // other role's waits on its commits therefore end.  The expanders
         // arrive for a K block only after they saw its stage's TMA
         // transaction complete, so the barrier covers both operands.
-        if (leader) {
-            const uint64_t qdesc0 = sw128_desc(sbase + kActOff);          // stage 0; + s * (kActStage >> 4)
-            const uint32_t a_tm0 = tmem_base + uint32_t(kACol0);          // A buffer 0; + 32 * a
-            const uint32_t empty0 = smem_u32(&empty_bar[0]), aempty0 = smem_u32(&aempty_bar[0]);
-            int it = 0, tcount = 0, s = 0, a = 0;
-            for (int ti = tbeg; ti < tend; ++ti, ++tcount) {
-                const TileRef tr = decode_tile(p, p.tiles[ti]);
-                const GemmProblem &P = p.prob[tr.g];
-                const int kblocks = P.kb;
-                const uint32_t idesc = idesc_i8((tile_tokens(P, tr.t_tile) + 15) & ~15);
-                const int b = tcount & 1;
-                if (tcount >= 2) nb_sync(kNbAcc0 + uint32_t(b));   // both epilogues drained tile tcount-2
-                if (ctrace && lane == 0 && tcount < 16) ctrace[24 + tcount] = clock_ordered();
-                const uint32_t d_tmem = tmem_base + uint32_t(b * kBT);
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    nb_sync(kNbAbuf0 + uint32_t(a));                   // both CTAs' A buffer a hold K block it
-                    if (lane == 0) stamp(it, 2);
-                    tc_fence_after();
-                    if (lane == 0)
-                        mma_kblock(d_tmem, a_tm0 + 32u * uint32_t(a), qdesc0 + uint64_t(s) * (kActStage >> 4),
-                                   idesc, kb > 0 ? 1u : 0u, empty0 + 8u * uint32_t(s), aempty0 + 8u * uint32_t(a));
-                    __syncwarp();
-                    if (lane == 0) stamp(it, 3);
-                    s = (s + 1 == kStages) ? 0 : s + 1;
-                    a = (a + 1) & (kABufs - 1);
-                }
-                if (lane == 0) mma_commit_pair(smem_u32(&accf_bar[b]));
+        const uint64_t qdesc0 = sw128_desc(sbase + kActOff);          // stage 0; + s * (kActStage >> 4)
+        const uint32_t a_tm0 = tmem_base + uint32_t(kACol0);          // A buffer 0; + 32 * a
+        const uint32_t empty0 = smem_u32(&empty_bar[0]), aempty0 = smem_u32(&aempty_bar[0]);
+        int it = 0, tcount = 0, s = 0, a = 0;
+        for (int ti = tbeg; ti < tend; ++ti, ++tcount) {
+            const TileRef tr = decode_tile(p, p.tiles[ti]);
+            const GemmProblem &P = p.prob[tr.g];
+            const int kblocks = P.kb;
+            const uint32_t idesc = idesc_i8((tile_tokens(P, tr.t_tile) + 15) & ~15);
+            const int b = tcount & 1;
+            if (tcount >= 2) nb_sync(kNbAcc0 + uint32_t(b));   // the epilogue drained tile tcount-2
+            if (ctrace && lane == 0 && tcount < 16) ctrace[24 + tcount] = clock64();
+            const uint32_t d_tmem = tmem_base + uint32_t(b * kBT);
+            for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                nb_sync(kNbAbuf0 + uint32_t(a));                   // A buffer a holds K block it
+                if (lane == 0) stamp(it, 2);
+                tc_fence_after();
+                if (lane == 0)
+                    mma_kblock(d_tmem, a_tm0 + 32u * uint32_t(a), qdesc0 + uint64_t(s) * (kActStage >> 4), idesc,
+                               kb > 0 ? 1u : 0u, empty0 + 8u * uint32_t(s), aempty0 + 8u * uint32_t(a));
                 __syncwarp();
+                if (lane == 0) stamp(it, 3);
+                s = (s + 1 == kStages) ? 0 : s + 1;
+                a = (a + 1) & (kABufs - 1);
             }
-            // the epilogues' arrivals for the last two tiles
-            for (int t = (tcount > 2 ? tcount - 2 : 0); t < tcount; ++t) nb_sync(kNbAcc0 + uint32_t(t & 1));
-            if (tcount > 0 && lane == 0) {
-                // all MMAs are complete (and their commits delivered) before
-                // either CTA frees TMEM or exits
-                mma_commit_local(smem_u32(&drain_bar));
-                mbar_wait(smem_u32(&drain_bar), 0, kDrainWaitLimit);
-            }
+            if (lane == 0) mma_commit(smem_u32(&accf_bar[b]));
             __syncwarp();
         }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ relay
-        // First CTA only: walks the MMA warp's sequence of named-barrier
-        // phases and, for each, waits for the second CTA's matching remote
-        // arrivals (its expanders for an A buffer, its epilogue for an
-        // accumulator), then arrives.  Those arrivals come once per phase
-        // whatever happens, so these waits end; after the long limit (a bug)
-        // it raises the flag and arrives anyway.
-        if (leader) {
-            int it = 0, tcount = 0;
-            for (int ti = tbeg; ti < tend; ++ti, ++tcount) {
-                const int kblocks = p.prob[decode_tile(p, p.tiles[ti]).g].kb;
-                const int b = tcount & 1;
-                if (tcount >= 2) {
-                    if (!warp_wait_progress(smem_u32(&peer_drained_bar[b]), ((tcount - 2) >> 1) & 1, long_limit,
-                                            true) &&
-                        lane == 0)
-                        fail();
-                    nb_arrive(kNbAcc0 + uint32_t(b));
-                }
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const int a = it % kABufs;
-                    if (!warp_wait_progress(smem_u32(&peer_ready_bar[a]), (it / kABufs) & 1, long_limit, true) &&
-                        lane == 0)
-                        fail();
-                    if (lane == 0) stamp(it, 1);
-                    nb_arrive(kNbAbuf0 + uint32_t(a));
-                }
-            }
-            for (int t = (tcount > 2 ? tcount - 2 : 0); t < tcount; ++t) {
-                if (!warp_wait_progress(smem_u32(&peer_drained_bar[t & 1]), (t >> 1) & 1, long_limit, true) &&
-                    lane == 0)
-                    fail();
-                nb_arrive(kNbAcc0 + uint32_t(t & 1));
-            }
+        // the epilogue's arrivals for the last two tiles
+        for (int t = (tcount > 2 ? tcount - 2 : 0); t < tcount; ++t) nb_sync(kNbAcc0 + uint32_t(t & 1));
+        if (tcount > 0 && lane == 0) {
+            // all MMAs this warp issued are complete before TMEM is freed
+            mma_commit(smem_u32(&drain_bar));
+            mbar_wait(smem_u32(&drain_bar), 0, kDrainWaitLimit);
         }
+        __syncwarp();
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------- expanders
-        // Every K block of the group ends with one arrival for its A buffer,
-        // in order, also after a failed wait (the work is then skipped): in
-        // the first CTA at the named barrier, in the second on the first
-        // CTA's peer_ready barrier (relayed).  Before writing a buffer again
-        // the group waits for the MMA warp's commit of its previous use, so
-        // it never arrives twice in one phase.
+        // Every K block of the group ends with one arrival at its A buffer's
+        // named barrier, in order, also after a failed wait (the work is then
+        // skipped): the MMA warp waits there without a limit.  Before writing
+        // a buffer again the group waits for the MMA warp's commit of its
+        // previous use, so it can never arrive twice in one barrier phase.
         const int grp = (warp - kExpandWarp0) / kExpandGroupWarps;
         const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
-        const int row = 32 * quad + lane;                // weight row of this CTA's half
+        const int row = 32 * quad + lane;                // weight row of the tile
         const uint32_t lane_addr = uint32_t(32 * quad) << 16;
         int it = 0;
         bool aborted = false;
@@ -618,20 +485,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (leader) {
-                    nb_arrive(kNbAbuf0 + uint32_t(a));
-                } else if (lane == 0) {
-                    remote_arrive(smem_u32(&peer_ready_bar[a]), 0);
-                }
+                nb_arrive(kNbAbuf0 + uint32_t(a));
                 if (lane == 0) stamp(it, 12 + quad);
             }
         }
     } else {
         // -------------------------------------------------------- epilogue
-        // One arrival per tile (first CTA: named barrier; second CTA: the
-        // first CTA's peer_drained barrier, relayed), in order, after the MMA
-        // warp's commit of that tile, so never twice in one phase; outputs
-        // are skipped once the launch has failed.
+        // One arrival per tile at the accumulator's named barrier, in order,
+        // after the MMA warp's commit of that tile (so never twice in one
+        // phase); the outputs are skipped once the launch has failed.
         const int quad = warp & 3;                       // TMEM lanes 32*quad .. 32*quad+31
         const uint32_t lane_addr = uint32_t(32 * quad) << 16;
         int tcount = 0;
@@ -657,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (!live && lane == 0) fail();
             live = __shfl_sync(0xffffffffu, (live && *abort_flag == 0) ? 1 : 0, 0) != 0;
             tc_fence_after();
-            const int f = tr.f_tile * kPairF + int(rank) * kBF + 32 * quad + lane;
+            const int f = tr.f_tile * kBF + 32 * quad + lane;
             const bool f_ok = f < n;
             const uint32_t taddr = tmem_base + lane_addr + uint32_t(b * kBT);
             if (live) {
@@ -667,7 +529,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     if (c0 >= nt) break;
                     uint32_t v[32];
                     tmem_ld32(taddr + uint32_t(c0), v);
-                    if (ctrace && quad == 0 && lane == 0 && tcount < 2) ctrace[40 + 16 * tcount + 2 * c] = clock_ordered();
+                    if (ctrace && quad == 0 && lane == 0 && tcount < 2) ctrace[40 + 16 * tcount + 2 * c] = clock64();
                     // dequantise all 32 in place first (straight-line code, so the
                     // shuffle -> convert -> multiply chains overlap), then store;
                     // a per-element branch here would serialise those chains
@@ -699,31 +561,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                 if (c0 + j < nt) yc[size_t(j) * size_t(n)] = __uint_as_float(v[j]);
                         }
                     }
-                    if (ctrace && quad == 0 && lane == 0 && tcount < 2) ctrace[41 + 16 * tcount + 2 * c] = clock_ordered();
+                    if (ctrace && quad == 0 && lane == 0 && tcount < 2) ctrace[41 + 16 * tcount + 2 * c] = clock64();
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (leader) {
-                nb_arrive(kNbAcc0 + uint32_t(b));
-            } else if (lane == 0) {
-                remote_arrive(smem_u32(&peer_drained_bar[b]), 0);
-            }
-            if (ctrace && tid == 32 * kEpiWarp0 && tcount < 16) ctrace[8 + tcount] = clock_ordered();
+            nb_arrive(kNbAcc0 + uint32_t(b));
+            if (ctrace && tid == 32 * kEpiWarp0 && tcount < 16) ctrace[8 + tcount] = clock64();
         }
     }
 
-    // neither CTA frees TMEM or exits while the other may still use its
-    // barriers, shared memory or TMEM
     tc_fence_before();
-    cluster_sync();
+    __syncthreads();
     tc_fence_after();
     if (ctrace && tid == 0) {
-        ctrace[2] = clock_ordered();
+        ctrace[2] = clock64();
         ctrace[4] = globaltimer();
     }
     if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
 }
 
@@ -745,8 +601,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 gemm_encode_fn()
 bool gemm_available() { return true; }
 
 // One or more grouped launches over `count` (<= kMaxGroup) problems sharing
-// the token count m.  Tiles are dealt heaviest-first to the least-loaded SM
-// pair (cost = MMA work of the tile's K loop plus a fixed epilogue share), so
+// the token count m.  Tiles are dealt heaviest-first to the least-loaded CTA
+// (cost = MMA work of the tile's K loop plus a fixed epilogue share), so
 // layers of different K balance inside one persistent launch.
 cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
                                 const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
@@ -771,7 +627,7 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
         {
             const cuuint64_t dims[2] = {cuuint64_t(128 * kb), cuuint64_t(m)};
             const cuuint64_t strides[1] = {cuuint64_t(128 * kb)};
-            const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kHalfT)};
+            const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kBT)};
             if (enc(&P.tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(xq[g]), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -794,7 +650,7 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
         P.n = int32_t(w[g].n);
         P.kb = int32_t(kb);
         P.tiles_t = tiles_t;
-        P.tiles_f = int32_t((w[g].n + kPairF - 1) / kPairF);
+        P.tiles_f = int32_t((w[g].n + kBF - 1) / kBF);
         P.tile0 = tile0;
         for (int ft = 0; ft < P.tiles_f; ++ft)
             for (int tt = 0; tt < tiles_t; ++tt) {
@@ -824,9 +680,8 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
     static thread_local std::vector<long long> load;
     for (size_t c0 = 0; c0 < all.size(); c0 += kMaxGemmTiles) {
         const int n = int(std::min<size_t>(kMaxGemmTiles, all.size() - c0));
-        const int G = std::min(std::min(sm_count / 2, kMaxGemmPairs), n);   // SM pairs
-        if (G < 1) return cudaErrorInvalidConfiguration;
-        // least-loaded pair first (loads are small integers: linear scan)
+        const int G = std::min(std::min(sm_count, kMaxGemmCtas), n);
+        // least-loaded CTA first (loads are small integers: linear scan)
         load.assign(G, 0);
         owner.assign(n, 0);
         count_of.assign(G, 0);
@@ -838,15 +693,14 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
             owner[i] = best;
             ++count_of[best];
         }
-        p.pair_off[0] = 0;
-        for (int c = 0; c < G; ++c) p.pair_off[c + 1] = p.pair_off[c] + count_of[c];
+        p.cta_off[0] = 0;
+        for (int c = 0; c < G; ++c) p.cta_off[c + 1] = p.cta_off[c] + count_of[c];
         fill.assign(G, 0);
         for (int i = 0; i < n; ++i) {
             const int c = owner[i];
-            p.tiles[p.pair_off[c] + fill[c]++] = all[c0 + i].id;
+            p.tiles[p.cta_off[c] + fill[c]++] = all[c0 + i].id;
         }
-        // grid = 2 CTAs per pair; the cluster shape (2, 1, 1) is compiled in
-        gemm_i2_kernel<<<2 * G, kGemmThreads, kGemmSmem, st>>>(p);
+        gemm_i2_kernel<<<G, kGemmThreads, kGemmSmem, st>>>(p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
