@@ -223,13 +223,23 @@ def _barrier():
 
 
 def _max_over_ranks(v):
+    """The slowest rank's value (every rank gets it).  One process per GPU
+    over NCCL in a bench run; the tensor lives where the backend wants it."""
     import torch
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
     return v
+
+
+def whole_job_rate(world, units_per_rank, max_ms):
+    """Units per second of the whole job: every rank processes
+    `units_per_rank` units per step (replicas, weak scaling), and the job's
+    step time is the slowest rank's."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 def run_gpu(args):
@@ -274,7 +284,7 @@ def run_gpu(args):
     total_ms = _max_over_ranks(total_ms)
     kern_ms = _max_over_ranks(statistics.mean(per))
     ms_step = total_ms / args.steps
-    tok_s = world * m / (ms_step * 1e-3)
+    tok_s = whole_job_rate(world, m, ms_step)
 
     # end to end through the C ABI: H2D inputs, stack call, D2H outputs per step
     e2e = None
@@ -290,7 +300,7 @@ def run_gpu(args):
         e_total, _ = time_device(e2e_step, max(args.steps // 2, 10), args.warmup, stream)
         e_total = _max_over_ranks(e_total)
         e_steps = max(args.steps // 2, 10)
-        e2e = {"value": world * m / (e_total / e_steps * 1e-3), "unit": "tokens/s",
+        e2e = {"value": whole_job_rate(world, m, e_total / e_steps), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_host.nbytes), "d2h_bytes_per_step": int(y_dev.numel() * 4)}
 
     peak, peak_kind, peaks = _peaks()
@@ -315,7 +325,7 @@ def run_gpu(args):
             t2, per2 = time_device(g2.replay, 50, 5, stream)
             t2 = _max_over_ranks(t2)
             k2 = _max_over_ranks(statistics.mean(per2))
-            sweep[str(ms)] = {"tokens_per_s": round(world * ms / (t2 / 50 * 1e-3), 1),
+            sweep[str(ms)] = {"tokens_per_s": round(whole_job_rate(world, ms, t2 / 50), 1),
                               "weight_gbs": round(stack_bytes / (k2 * 1e-3) / 1e9, 1)}
 
     prefill = None
@@ -418,7 +428,7 @@ def run_prefill(dev, stream, flags, world):
     _, _, peaks = _peaks()
     bf16 = float(peaks.get("bf16_tflops", 1590.0))
     peak = 2.0 * bf16          # int8 dense = 2 x bf16 dense (nominal 4.5 vs 2.25 PFLOP/s)
-    tops = world * PREFILL_OPS / (tg * 1e-3) / 1e12
+    tops = whole_job_rate(world, PREFILL_OPS, tg) / 1e12
     return {"workload": "M=2048 tokens x the seven decoder-layer shapes, int8 activations x ternary weights",
             "ops_per_step": PREFILL_OPS, "ms_per_step": round(tg, 5), "tops": round(tops, 1),
             "roofline": {"bound": "tensor", "achieved": round(tops / world, 1), "peak": round(peak, 1),
