@@ -21,6 +21,7 @@ for _name, _args, _ret in [
     ("oracle_kpad", [_i64], _i64),
     ("oracle_quant_act", [_P, _i64, _i64, _P, _P], _C.c_int),
     ("oracle_pack", [_P, _i64, _i64, _P], _C.c_int),
+    ("oracle_absmean_ternary", [_P, _i64, _i64, _P, _P], _C.c_int),
     ("oracle_unpack", [_P, _i64, _i64, _P], None),
     ("oracle_unpack_misread64", [_P, _i64, _i64, _P], None),
     ("oracle_ternary_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
@@ -60,6 +61,16 @@ def quant_act(x):
     s = _np.empty((m,), _np.float32)
     st = _lib.oracle_quant_act(_ptr(x), m, k, _ptr(q), _ptr(s))
     return q, s, st
+
+
+def absmean_ternary(W):
+    """W fp32 [n,k] -> (w int8 [n,k] in {-1,0,1}, scale fp32, status) (reading R5)."""
+    W = _c(W, _np.float32)
+    n, k = W.shape
+    w = _np.empty((n, k), _np.int8)
+    sc = _np.zeros((1,), _np.float32)
+    st = _lib.oracle_absmean_ternary(_ptr(W), n, k, _ptr(w), _ptr(sc))
+    return w, _np.float32(sc[0]), st
 
 
 def pack(w):

@@ -53,6 +53,41 @@ int oracle_quant_act(const float *x, int64_t m, int64_t k, int8_t *q, float *s_a
     return status;
 }
 
+/* R5 -- absmean ternary quantiser, written from its definition: one pass for
+ * the mean of |W| (fp64 sum in row-major order, one rounding to fp32), one
+ * pass for the codes (fp32 divide, fp32 rint, clamp to [-1, 1]). */
+int oracle_absmean_ternary(const float *W, int64_t n, int64_t k, int8_t *w, float *scale)
+{
+    const int64_t total = n * k;
+    double sum = 0.0;
+    int finite = 1;
+    for (int64_t i = 0; i < total; ++i) {
+        if (!isfinite(W[i])) {
+            finite = 0;
+            break;
+        }
+        sum += fabs((double)W[i]);
+    }
+    if (!finite || total == 0) {
+        for (int64_t i = 0; i < total; ++i) w[i] = 0;
+        *scale = 0.0f;
+        return finite ? ORACLE_OK : ORACLE_NONFINITE;
+    }
+    const float s = (float)(sum / (double)total);
+    *scale = s;
+    for (int64_t i = 0; i < total; ++i) {
+        if (s == 0.0f) {
+            w[i] = 0;
+            continue;
+        }
+        float v = rintf(W[i] / s);        /* one rounded fp32 quotient, half to even */
+        if (v > 1.0f) v = 1.0f;
+        if (v < -1.0f) v = -1.0f;
+        w[i] = (int8_t)(int)v;
+    }
+    return ORACLE_OK;
+}
+
 /* Position of element k inside a packed row (R2): byte index and bit shift. */
 static int64_t code_byte(int64_t k) { return 32 * (k / 128) + (k % 32); }
 static int code_shift(int64_t k) { return (int)(2 * ((k % 128) / 32)); }

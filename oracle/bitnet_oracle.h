@@ -29,6 +29,13 @@
  *  R4 linear: acc[m,n] = sum_{k<K} q[m,k]*w[n,k], exact integer;
  *       y[m,n] = acc[m,n] * s_act[m] * s_w evaluated in fp64 (the oracle's
  *       reference value); the fp32 form ((float)acc*s_act)*s_w is also given.
+ *  R5 absmean weight quantiser (the ternary weights of §2.2.2 come from a
+ *       full-precision tensor by the BitNet b1.58 recipe the report cites but
+ *       does not print; plainest reading): scale = mean over all n*k elements
+ *       of |W|, summed in fp64 and rounded once to fp32; w = clamp(rint(W /
+ *       scale), -1, 1) with the division and the rounding in fp32 (rounding
+ *       half to even).  An all-zero tensor gives scale 0 and w = 0; a tensor
+ *       holding NaN/Inf gives scale 0, w = 0 and ORACLE_NONFINITE.
  */
 #ifndef BITNET_ORACLE_H
 #define BITNET_ORACLE_H
@@ -56,6 +63,10 @@ int oracle_quant_act(const float *x, int64_t m, int64_t k, int8_t *q, float *s_a
 /* R2/R3: w int8 [n,k] -> packed [n, 32*blocks].  A value outside {-1,0,+1}
  * is stored as weight 0 and ORACLE_NOT_TERNARY is returned. */
 int oracle_pack(const int8_t *w, int64_t n, int64_t k, uint8_t *packed);
+
+/* R5: W fp32 [n,k] -> ternary w int8 [n,k] and the per-tensor scale.
+ * Returns ORACLE_NONFINITE if W held NaN or Inf. */
+int oracle_absmean_ternary(const float *W, int64_t n, int64_t k, int8_t *w, float *scale);
 
 /* Inverse of oracle_pack: packed [n, 32*blocks] -> w int8 [n,k]. */
 void oracle_unpack(const uint8_t *packed, int64_t n, int64_t k, int8_t *w);

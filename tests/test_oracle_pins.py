@@ -293,3 +293,77 @@ def test_linear_rows_sampled_equals_full():
     a2, y2, _ = oracle.linear_rows(x, p, n, k, 0.07, idx)
     np.testing.assert_array_equal(a2, acc[:, idx])
     np.testing.assert_array_equal(y2, y64[:, idx])
+
+
+# ------------------------------------------------------ absmean quantiser (R5)
+
+def _read_absmean_golden():
+    cases, cur = [], {}
+    for line in open(os.path.join(GOLDEN, "absmean_small.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, val = line.split(":", 1)
+        rows = [[float(v) for v in r.split()] for r in val.split("|")] if key != "s" else float(val)
+        cur[key] = rows
+        if key == "s":
+            cases.append(cur)
+            cur = {}
+    return cases
+
+
+def test_absmean_golden_examples():
+    cases = _read_absmean_golden()
+    assert len(cases) == 4
+    for c in cases:
+        W = np.array(c["rows"], np.float32)
+        w, s, st = oracle.absmean_ternary(W)
+        assert st == oracle.OK
+        np.testing.assert_array_equal(w, np.array(c["w"], np.int8))
+        assert s == np.float32(c["s"])
+
+
+@pytest.mark.parametrize("p_nonzero", [1.0, 0.75, 0.5, 0.25])
+def test_absmean_closed_form_scaled_ternary(p_nonzero):
+    """W = c * T with T ternary and a known count of nonzeros: mean|W| = c * p
+    exactly, W / scale = T / p has magnitude >= 1 wherever T != 0, so the
+    codes give back T."""
+    rng = np.random.default_rng(int(p_nonzero * 100))
+    n, k = 16, 256
+    nz = int(p_nonzero * n * k)
+    T = np.zeros(n * k, np.int8)
+    T[:nz] = rng.choice([-1, 1], nz)
+    rng.shuffle(T)
+    T = T.reshape(n, k)
+    c = np.float32(0.03125)
+    w, s, st = oracle.absmean_ternary(c * T.astype(np.float32))
+    assert st == oracle.OK
+    assert s == np.float32(c * nz / (n * k))
+    np.testing.assert_array_equal(w, T)
+
+
+def test_absmean_power_of_two_equivariance_and_invariants():
+    """Scaling W by 2^e scales the mean exactly and leaves every quotient, so
+    every code, unchanged; on random W the codes are ternary, carry W's sign,
+    are 0 exactly where |W| / scale <= 1/2 and 1 in magnitude elsewhere."""
+    rng = np.random.default_rng(77)
+    W = (rng.standard_normal((48, 520)) * 0.02).astype(np.float32)
+    w, s, st = oracle.absmean_ternary(W)
+    assert st == oracle.OK and s > 0
+    for e in (-3, 5):
+        w2, s2, _ = oracle.absmean_ternary(W * np.float32(2.0 ** e))
+        assert s2 == np.float32(s * 2.0 ** e)
+        np.testing.assert_array_equal(w2, w)
+    assert set(np.unique(w)) <= {-1, 0, 1}
+    assert (np.sign(w[w != 0]) == np.sign(W[w != 0])).all()
+    ratio = np.abs(W / s)          # the fp32 quotient the codes are decided on
+    assert (w[ratio < 0.5] == 0).all() and (np.abs(w[ratio > 0.5]) == 1).all()
+
+
+def test_absmean_nonfinite_tensor():
+    W = np.ones((3, 7), np.float32)
+    for bad in (np.nan, np.inf, -np.inf):
+        W2 = W.copy()
+        W2[1, 4] = bad
+        w, s, st = oracle.absmean_ternary(W2)
+        assert st == oracle.NONFINITE and s == 0.0 and not w.any()
