@@ -331,6 +331,7 @@ def run_gpu(args):
     prefill = None
     if not args.no_prefill:
         prefill = run_prefill(dev, stream, flags, world)
+    qpack = run_quantize_pack(dev, stream, flags, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -357,6 +358,7 @@ def run_gpu(args):
             "clocks": clk,
             "m_sweep": sweep,
             "prefill": prefill,
+            "quantize_pack": qpack,
         }
         print(json.dumps(line))
     if world > 1:
@@ -436,6 +438,52 @@ def run_prefill(dev, stream, flags, world):
                          "peak_kind": "measured bf16 cuBLAS burst (MEASURED_PEAKS.json) x 2 (int8:bf16 dense ratio)"},
             "quant_ms_per_step": round(tq, 5), "per_shape": per_shape,
             "kernel": "gemm_i2_kernel (tcgen05.mma kind::i8, weights expanded into TMEM as A, activations as B from shared memory, 128 features x 192 tokens x 128 tiles, one grouped launch)"}
+
+
+def run_quantize_pack(dev, stream, flags, world):
+    """Load-time absmean quantise + pack of one decoder layer's seven fp32
+    weight tensors (187 MB of fp32, larger than L2), graph-replayed: three
+    launches per tensor.  Algorithmic bytes: 4 B read + 1/4 B written per
+    weight; the kernel reads each tensor twice, the second time mostly from
+    L2 (a tensor is at most 55 MB)."""
+    import torch
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import synth
+
+    ws = torch.empty(tw2.quantize_pack_workspace_bytes(), dtype=torch.uint8, device=dev)
+    scales = torch.empty(len(synth.LAYER_SHAPES), dtype=torch.float32, device=dev)
+    work, weights = [], 0
+    for i, (name, n, k) in enumerate(synth.LAYER_SHAPES):
+        g = torch.Generator(device=dev)
+        g.manual_seed(synth.seed_for(5, i))
+        W = torch.randn((n, k), generator=g, device=dev, dtype=torch.float32) * 0.02
+        pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
+        work.append((W, pk, scales[i:i + 1]))
+        weights += n * k
+
+    def step():
+        for W, pk, sc in work:
+            tw2.quantize_pack(W, pk, sc, ws, flags=flags)
+
+    step()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        step()
+    steps = 20
+    t, _ = time_device(gr.replay, steps, 3, stream)
+    t = _max_over_ranks(t) / steps
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"device flags {int(flags.item())} in the quantize_pack run")
+    hbm, _, _ = _peaks()
+    alg = 4.25 * weights
+    gbs = alg / (t * 1e-3) / 1e9
+    return {"workload": "absmean quantise + pack of one decoder layer's seven fp32 weight tensors "
+                        "(%d weights, %.1f MB fp32 > L2)" % (weights, 4 * weights / 1e6),
+            "ms_per_step": round(t, 5), "launches_per_step": 3 * len(work),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes_per_weight": 4.25},
+            "kernels": "absmean_partial_kernel, absmean_scale_kernel, absmean_pack_kernel"}
 
 
 def build_stack_views(m, dev, tws, layers=28):

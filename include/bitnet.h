@@ -139,6 +139,35 @@ BITNET_API int64_t bitnet_kpad(int64_t k);
 BITNET_API bitnet_status bitnet_pack_ternary(const int8_t *w, int64_t n, int64_t k,
                                   uint8_t *packed, int32_t *d_flags, void *stream);
 
+/* Workspace bytes bitnet_quantize_pack needs (a fixed 4096). */
+BITNET_API size_t bitnet_quantize_pack_workspace_bytes(void);
+
+/*
+ * Absmean ternary quantiser fused with the pack: full-precision weights ->
+ * the 2-bit format above + one per-tensor scale (the ternary weights and
+ * per-tensor scale of the technical report §2.2.2; the rounding rule is
+ * the absmean recipe of the BitNet b1.58 work the report builds on, taken as):
+ *   scale = mean |W| over all n*k elements, summed in fp64 and rounded once
+ *           to fp32;
+ *   w     = clamp(rint(W / scale), -1, +1), quotient in fp32 (correctly
+ *           rounded), rint half to even;
+ *   an all-zero W gives scale 0 and every w = 0.
+ *   w          device fp32 [n, k], 4-byte aligned
+ *   packed     device, [n, 32*ceil(k/128)] bytes, 16-byte aligned; fully written
+ *   d_scale    device fp32 [1], receives scale (w_scale of the linear call)
+ *   workspace  device, 8-byte aligned, >= bitnet_quantize_pack_workspace_bytes()
+ *              bytes, owned by the caller; must not be reused by another call
+ *              until this one has completed on `stream`
+ *   d_flags    device int32 or NULL
+ * A non-finite element sets scale 0 and every w = 0 and raises
+ * BITNET_FLAG_NONFINITE.  The result does not depend on the device or the
+ * launch: the fp64 partial sums use a fixed grid and a fixed order.
+ * Load-time operation (three kernel launches on `stream`).
+ */
+BITNET_API bitnet_status bitnet_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed,
+                                              float *d_scale, void *workspace, size_t workspace_bytes,
+                                              int32_t *d_flags, void *stream);
+
 /* Inverse of bitnet_pack_ternary (test and inspection aid):
  *   packed device [n, 32*ceil(k/128)] -> w device int8 [n, k]. */
 BITNET_API bitnet_status bitnet_unpack_ternary(const uint8_t *packed, int64_t n, int64_t k,

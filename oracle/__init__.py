@@ -22,6 +22,7 @@ for _name, _args, _ret in [
     ("oracle_quant_act", [_P, _i64, _i64, _P, _P], _C.c_int),
     ("oracle_pack", [_P, _i64, _i64, _P], _C.c_int),
     ("oracle_absmean_ternary", [_P, _i64, _i64, _P, _P], _C.c_int),
+    ("oracle_ternary_round", [_P, _i64, _f32, _P], None),
     ("oracle_unpack", [_P, _i64, _i64, _P], None),
     ("oracle_unpack_misread64", [_P, _i64, _i64, _P], None),
     ("oracle_ternary_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
@@ -71,6 +72,14 @@ def absmean_ternary(W):
     sc = _np.zeros((1,), _np.float32)
     st = _lib.oracle_absmean_ternary(_ptr(W), n, k, _ptr(w), _ptr(sc))
     return w, _np.float32(sc[0]), st
+
+
+def ternary_round(W, scale):
+    """Codes of W fp32 [n,k] at a given fp32 scale (second pass of reading R5)."""
+    W = _c(W, _np.float32)
+    w = _np.empty(W.shape, _np.int8)
+    _lib.oracle_ternary_round(_ptr(W), W.size, _np.float32(scale), _ptr(w))
+    return w
 
 
 def pack(w):

@@ -53,9 +53,25 @@ int oracle_quant_act(const float *x, int64_t m, int64_t k, int8_t *q, float *s_a
     return status;
 }
 
+/* R5, second pass -- the ternary codes at a given scale s: fp32 divide, fp32
+ * rint (half to even), clamp to [-1, 1]; s == 0 gives every code 0. */
+void oracle_ternary_round(const float *W, int64_t total, float s, int8_t *w)
+{
+    for (int64_t i = 0; i < total; ++i) {
+        if (s == 0.0f) {
+            w[i] = 0;
+            continue;
+        }
+        float v = rintf(W[i] / s);        /* one rounded fp32 quotient, half to even */
+        if (v > 1.0f) v = 1.0f;
+        if (v < -1.0f) v = -1.0f;
+        w[i] = (int8_t)(int)v;
+    }
+}
+
 /* R5 -- absmean ternary quantiser, written from its definition: one pass for
  * the mean of |W| (fp64 sum in row-major order, one rounding to fp32), one
- * pass for the codes (fp32 divide, fp32 rint, clamp to [-1, 1]). */
+ * pass for the codes at that scale. */
 int oracle_absmean_ternary(const float *W, int64_t n, int64_t k, int8_t *w, float *scale)
 {
     const int64_t total = n * k;
@@ -75,16 +91,7 @@ int oracle_absmean_ternary(const float *W, int64_t n, int64_t k, int8_t *w, floa
     }
     const float s = (float)(sum / (double)total);
     *scale = s;
-    for (int64_t i = 0; i < total; ++i) {
-        if (s == 0.0f) {
-            w[i] = 0;
-            continue;
-        }
-        float v = rintf(W[i] / s);        /* one rounded fp32 quotient, half to even */
-        if (v > 1.0f) v = 1.0f;
-        if (v < -1.0f) v = -1.0f;
-        w[i] = (int8_t)(int)v;
-    }
+    oracle_ternary_round(W, total, s, w);
     return ORACLE_OK;
 }
 

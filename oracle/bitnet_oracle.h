@@ -66,6 +66,9 @@ int oracle_pack(const int8_t *w, int64_t n, int64_t k, uint8_t *packed);
 
 /* R5: W fp32 [n,k] -> ternary w int8 [n,k] and the per-tensor scale.
  * Returns ORACLE_NONFINITE if W held NaN or Inf. */
+/* R5, second pass: codes clamp(rint(W / s), -1, 1) for a given fp32 scale s
+ * (fp32 quotient, half to even); s == 0 gives 0 everywhere. */
+void oracle_ternary_round(const float *W, int64_t total, float s, int8_t *w);
 int oracle_absmean_ternary(const float *W, int64_t n, int64_t k, int8_t *w, float *scale);
 
 /* Inverse of oracle_pack: packed [n, 32*blocks] -> w int8 [n,k]. */

@@ -8,6 +8,7 @@ from ._abi import (  # noqa: F401
     BitnetError, StackCall, TW, header_functions, kpad, linear, linear_q, linear_stack,
     linear_stack_noalloc, linear_q_grouped, GroupedCall,
     linear_workspace_bytes, load, make_tw, pack_ternary, packed_bytes, quant_act,
+    quantize_pack, quantize_pack_workspace_bytes,
     status_from_flags, unpack_ternary, version,
     FLAG_NONFINITE, FLAG_NOT_TERNARY, FLAG_TIMEOUT, GEMV_MAX_M, MAX_K, STACK_MAX,
 )

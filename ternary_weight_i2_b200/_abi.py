@@ -44,6 +44,8 @@ _SIGNATURES = {
     "bitnet_kpad": ([_I64], _I64),
     "bitnet_pack_ternary": ([_P, _I64, _I64, _P, _P, _P], C.c_int),
     "bitnet_unpack_ternary": ([_P, _I64, _I64, _P, _P], C.c_int),
+    "bitnet_quantize_pack_workspace_bytes": ([], C.c_size_t),
+    "bitnet_quantize_pack": ([_P, _I64, _I64, _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
     "bitnet_quant_act": ([_P, _I64, _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_linear_workspace_bytes": ([_I64, _I64], C.c_size_t),
     "bitnet_linear": ([_P, _I64, C.POINTER(TW), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
@@ -152,6 +154,19 @@ def pack_ternary(w, packed, flags=None, stream=None) -> None:
     n, k = w.shape
     _check(load().bitnet_pack_ternary(_ptr(w), n, k, _ptr(packed), _ptr(flags), _stream(stream)),
            "bitnet_pack_ternary")
+
+
+def quantize_pack_workspace_bytes() -> int:
+    return int(load().bitnet_quantize_pack_workspace_bytes())
+
+
+def quantize_pack(w, packed, scale, workspace, flags=None, stream=None) -> None:
+    """w: fp32 [n,k] device tensor -> packed uint8 [n, 32*ceil(k/128)] and the
+    absmean scale in the one-element fp32 device tensor ``scale``."""
+    n, k = w.shape
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().bitnet_quantize_pack(_ptr(w), n, k, _ptr(packed), _ptr(scale), _ptr(workspace), ws_bytes,
+                                       _ptr(flags), _stream(stream)), "bitnet_quantize_pack")
 
 
 def unpack_ternary(packed, n, k, w, stream=None) -> None:

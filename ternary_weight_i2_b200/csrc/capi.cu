@@ -20,6 +20,8 @@ cudaError_t launch_pack(const int8_t *w, int64_t n, int64_t k, uint8_t *packed, 
 cudaError_t launch_unpack(const uint8_t *packed, int64_t n, int64_t k, int8_t *w, cudaStream_t st);
 cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float *scale, int32_t *flags,
                          cudaStream_t st);
+cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
+                                 int32_t *flags, cudaStream_t st);
 bool gemm_available();
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
                         int32_t *acc, int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count,
@@ -532,6 +534,26 @@ bitnet_status bitnet_pack_ternary(const int8_t *w, int64_t n, int64_t k, uint8_t
     if (s != BITNET_OK) return s;
     cudaError_t e = launch_pack(w, n, k, packed, d_flags, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "pack launch");
+}
+
+size_t bitnet_quantize_pack_workspace_bytes(void) { return 4096; }
+
+bitnet_status bitnet_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *d_scale,
+                                   void *workspace, size_t workspace_bytes, int32_t *d_flags, void *stream)
+{
+    if (!w || !packed || !d_scale || !workspace) return fail(BITNET_ERR_INVALID_ARG, "quantize_pack: NULL pointer");
+    if (n < 1 || k < 1 || k > BITNET_MAX_K)
+        return fail(BITNET_ERR_INVALID_ARG, "quantize_pack: bad sizes n=%lld k=%lld", (long long)n, (long long)k);
+    if (!aligned(w, 4) || !aligned(packed, 16) || !aligned(d_scale, 4) || !aligned(workspace, 8))
+        return fail(BITNET_ERR_INVALID_ARG, "quantize_pack: misaligned pointer");
+    if (workspace_bytes < bitnet_quantize_pack_workspace_bytes())
+        return fail(BITNET_ERR_WORKSPACE, "quantize_pack: workspace %zu < %zu bytes", workspace_bytes,
+                    bitnet_quantize_pack_workspace_bytes());
+    DevInfo dev;
+    bitnet_status s = check_device(&dev);
+    if (s != BITNET_OK) return s;
+    cudaError_t e = launch_quantize_pack(w, n, k, packed, d_scale, workspace, d_flags, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "quantize_pack launch");
 }
 
 bitnet_status bitnet_unpack_ternary(const uint8_t *packed, int64_t n, int64_t k, int8_t *w, void *stream)

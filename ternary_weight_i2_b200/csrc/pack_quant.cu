@@ -122,6 +122,127 @@ __global__ void __launch_bounds__(NT) quant_kernel(const float *__restrict__ x, 
     }
 }
 
+// ------------------------------------------------------------- absmean
+// Absmean ternary quantiser fused with the pack.  The ternary weights of the
+// report's §2.2.2 come from a full-precision tensor by a recipe the report
+// cites but does not print; the reading taken: scale = mean |W| over the
+// tensor, summed in fp64 and rounded once to fp32; w = clamp(rint(W /
+// scale), -1, 1) with the quotient and the rounding in fp32 (half to even);
+// an all-zero tensor gives scale 0 and w = 0; a non-finite element gives
+// scale 0, w = 0 and BITNET_FLAG_NONFINITE.
+//
+// Three launches, each deterministic: per-CTA fp64 partial sums of |W| over
+// a fixed grid (so the summation order, hence the scale, is the same on every
+// call and every device), one thread summing the partials in a fixed order,
+// and the quantise-and-pack pass.
+
+constexpr int kAbsmeanCtas = 256, kAbsmeanThreads = 256;
+
+struct AbsmeanScratch {
+    double partial[kAbsmeanCtas];
+    int32_t bad[kAbsmeanCtas];
+};
+static_assert(sizeof(AbsmeanScratch) <= 4096, "absmean workspace");
+
+__global__ void __launch_bounds__(kAbsmeanThreads) absmean_partial_kernel(const float *__restrict__ W, int64_t total,
+                                                                       AbsmeanScratch *scratch)
+{
+    __shared__ double wsum[kAbsmeanThreads / 32];
+    __shared__ int wbad[kAbsmeanThreads / 32];
+    double s = 0.0;
+    bool bad = false;
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    // eight loads in flight per thread; the adds keep the plain loop's order
+    for (; i + 7 * stride < total; i += 8 * stride) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = W[i + u * stride];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            bad |= !isfinite(v[u]);
+            s += fabs(double(v[u]));
+        }
+    }
+    for (; i < total; i += stride) {
+        const float v = W[i];
+        bad |= !isfinite(v);
+        s += fabs(double(v));
+    }
+    // fixed reduction tree: xor shuffles within the warp, then warps in order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const bool any_bad = __any_sync(0xffffffffu, bad);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        wsum[warp] = s;
+        wbad[warp] = any_bad ? 1 : 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        int b = 0;
+        for (int w = 0; w < kAbsmeanThreads / 32; ++w) {
+            t += wsum[w];
+            b |= wbad[w];
+        }
+        scratch->partial[blockIdx.x] = t;
+        scratch->bad[blockIdx.x] = b;
+    }
+}
+
+__global__ void absmean_scale_kernel(const AbsmeanScratch *scratch, int64_t total, float *scale, int32_t *flags)
+{
+    if (threadIdx.x != 0) return;
+    double t = 0.0;
+    int b = 0;
+    for (int i = 0; i < kAbsmeanCtas; ++i) {
+        t += scratch->partial[i];
+        b |= scratch->bad[i];
+    }
+    if (b) raise_flag(flags, BITNET_FLAG_NONFINITE);
+    *scale = (b || total == 0) ? 0.f : float(t / double(total));
+}
+
+// One thread per packed 32-bit word: bytes 4t .. 4t+3 of block j hold, in
+// field g, elements 128j + 32g + 4t + i (i = 0..3) -- four consecutive
+// weights per field, read by 8 consecutive threads as 128 contiguous bytes.
+__global__ void absmean_pack_kernel(const float *__restrict__ W, int64_t n, int64_t k, int64_t kb, bool vec4,
+                                    const float *__restrict__ scale, uint32_t *__restrict__ packed)
+{
+    const float s = *scale;
+    const int64_t row_words = 8 * kb, total = n * row_words;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+         idx += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = idx / row_words, wi = idx - r * row_words;
+        const int64_t j = wi >> 3, t = wi & 7;
+        const float *wr = W + r * k;
+        uint32_t out = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int64_t k0 = 128 * j + 32 * g + 4 * t;
+            float v[4];
+            if (vec4 && k0 + 3 < k) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(wr + k0));
+                v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[i] = k0 + i < k ? wr[k0 + i] : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t code = 1;   // weight 0: tails, and every weight when s == 0
+                if (k0 + i < k && s != 0.f) {
+                    const float q = fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -1.f), 1.f);
+                    code = uint32_t(int(q) + 1);
+                }
+                out |= code << (8 * i + 2 * g);
+            }
+        }
+        packed[idx] = out;
+    }
+}
+
 static int grid_for(int64_t work, int threads)
 {
     int64_t g = (work + threads - 1) / threads;
@@ -148,6 +269,20 @@ cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float
 {
     const int64_t kpad = 128 * ((k + 127) / 128);
     quant_kernel<256><<<unsigned(m), 256, 0, st>>>(x, m, k, kpad, xq, scale, flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
+                                 int32_t *flags, cudaStream_t st)
+{
+    const int64_t kb = (k + 127) / 128;
+    auto *scratch = static_cast<AbsmeanScratch *>(workspace);
+    absmean_partial_kernel<<<kAbsmeanCtas, kAbsmeanThreads, 0, st>>>(w, n * k, scratch);
+    absmean_scale_kernel<<<1, 32, 0, st>>>(scratch, n * k, scale, flags);
+    // float4 loads need every row start 16-byte aligned: W aligned and k % 4 == 0
+    const bool vec4 = (reinterpret_cast<uintptr_t>(w) & 15) == 0 && k % 4 == 0;
+    absmean_pack_kernel<<<grid_for(n * 8 * kb, 256), 256, 0, st>>>(w, n, k, kb, vec4, scale,
+                                                                  reinterpret_cast<uint32_t *>(packed));
     return cudaGetLastError();
 }
 

@@ -367,3 +367,20 @@ def test_absmean_nonfinite_tensor():
         W2[1, 4] = bad
         w, s, st = oracle.absmean_ternary(W2)
         assert st == oracle.NONFINITE and s == 0.0 and not w.any()
+
+
+def test_ternary_round_at_given_scale_hand_table():
+    """The second pass alone, at scale 2, against codes worked by hand from
+    clamp(rint(W / 2), -1, 1): quotients exactly +-0.5 round to 0 (half to
+    even), just above 0.5 to 1, +-1.5 to +-2 and clamp; scale 0 gives 0."""
+    W = np.array([[-3.1, -3.0, -1.0, -0.99, 0.0, 1.0, 1.0000001, 3.0, 100.0]], np.float32)
+    want = np.array([[-1, -1, 0, 0, 0, 0, 1, 1, 1]], np.int8)
+    np.testing.assert_array_equal(oracle.ternary_round(W, 2.0), want)
+    assert not oracle.ternary_round(W, 0.0).any()
+
+
+def test_absmean_codes_are_the_second_pass_at_its_own_scale():
+    rng = np.random.default_rng(78)
+    W = (rng.standard_normal((9, 301)) * 0.1).astype(np.float32)
+    w, s, _ = oracle.absmean_ternary(W)
+    np.testing.assert_array_equal(oracle.ternary_round(W, s), w)
