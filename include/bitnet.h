@@ -139,7 +139,7 @@ BITNET_API int64_t bitnet_kpad(int64_t k);
 BITNET_API bitnet_status bitnet_pack_ternary(const int8_t *w, int64_t n, int64_t k,
                                   uint8_t *packed, int32_t *d_flags, void *stream);
 
-/* Workspace bytes bitnet_quantize_pack needs (a fixed 4096). */
+/* Workspace bytes bitnet_quantize_pack needs (a fixed 16384). */
 BITNET_API size_t bitnet_quantize_pack_workspace_bytes(void);
 
 /*
@@ -162,7 +162,7 @@ BITNET_API size_t bitnet_quantize_pack_workspace_bytes(void);
  * A non-finite element sets scale 0 and every w = 0 and raises
  * BITNET_FLAG_NONFINITE.  The result does not depend on the device or the
  * launch: the fp64 partial sums use a fixed grid and a fixed order.
- * Load-time operation (three kernel launches on `stream`).
+ * Load-time operation (two kernel launches on `stream`).
  */
 BITNET_API bitnet_status bitnet_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed,
                                               float *d_scale, void *workspace, size_t workspace_bytes,

@@ -21,7 +21,7 @@ cudaError_t launch_unpack(const uint8_t *packed, int64_t n, int64_t k, int8_t *w
 cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float *scale, int32_t *flags,
                          cudaStream_t st);
 cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
-                                 int32_t *flags, cudaStream_t st);
+                                 int32_t *flags, int sm_count, cudaStream_t st);
 bool gemm_available();
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
                         int32_t *acc, int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count,
@@ -536,7 +536,7 @@ bitnet_status bitnet_pack_ternary(const int8_t *w, int64_t n, int64_t k, uint8_t
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "pack launch");
 }
 
-size_t bitnet_quantize_pack_workspace_bytes(void) { return 4096; }
+size_t bitnet_quantize_pack_workspace_bytes(void) { return 16384; }
 
 bitnet_status bitnet_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *d_scale,
                                    void *workspace, size_t workspace_bytes, int32_t *d_flags, void *stream)
@@ -552,7 +552,8 @@ bitnet_status bitnet_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t
     DevInfo dev;
     bitnet_status s = check_device(&dev);
     if (s != BITNET_OK) return s;
-    cudaError_t e = launch_quantize_pack(w, n, k, packed, d_scale, workspace, d_flags, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_quantize_pack(w, n, k, packed, d_scale, workspace, d_flags, dev.sm_count,
+                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "quantize_pack launch");
 }
 

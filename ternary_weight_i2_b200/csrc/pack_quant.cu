@@ -131,88 +131,139 @@ __global__ void __launch_bounds__(NT) quant_kernel(const float *__restrict__ x, 
 // an all-zero tensor gives scale 0 and w = 0; a non-finite element gives
 // scale 0, w = 0 and BITNET_FLAG_NONFINITE.
 //
-// Three launches, each deterministic: per-CTA fp64 partial sums of |W| over
-// a fixed grid (so the summation order, hence the scale, is the same on every
-// call and every device), one thread summing the partials in a fixed order,
-// and the quantise-and-pack pass.
+// Two launches, each deterministic.  The first writes per-CTA fp64 partial
+// sums of |W| over a fixed grid, so the summation order, hence the scale, is
+// the same on every call and every device.  The second has every CTA sum the
+// partials by the same fixed tree (each CTA finds the same scale; CTA 0
+// publishes it) and then quantises and packs.
+//
+// The rounding decision without a divide.  With s > 0 the code is 0 exactly
+// when rint(fl(|W| / s)) == 0, i.e. when fl(|W| / s) <= 1/2 (1/2 is even).
+// Rounding is monotone and the floats next to 1/2 are 1/2 - 2^-25 and
+// 1/2 + 2^-24, so fl(q) <= 1/2 exactly when the real quotient q <= 1/2 +
+// 2^-25 (the midpoint rounds to the even 1/2), i.e. |W| <= s * (1/2 + 2^-25).
+// That product has at most 49 significant bits and is exact in fp64, as is
+// |W|, so the fp64 comparison takes the same decision as the fp32 divide
+// followed by rint.  Any other quotient rounds to a nonzero integer and
+// clamps to sign(W).
 
-constexpr int kAbsmeanCtas = 256, kAbsmeanThreads = 256;
+constexpr int kAbsmeanCtas = 1024, kAbsmeanThreads = 256, kAbsmeanPackCtasPerSm = 4;
+constexpr double kHalfPlusHalfUlp = 0.5 + 0x1p-25;
 
 struct AbsmeanScratch {
     double partial[kAbsmeanCtas];
     int32_t bad[kAbsmeanCtas];
 };
-static_assert(sizeof(AbsmeanScratch) <= 4096, "absmean workspace");
+static_assert(sizeof(AbsmeanScratch) <= 16384, "absmean workspace");
 
-__global__ void __launch_bounds__(kAbsmeanThreads) absmean_partial_kernel(const float *__restrict__ W, int64_t total,
-                                                                       AbsmeanScratch *scratch)
+// Four consecutive elements 4u .. 4u+3 of the flattened tensor; positions
+// past the end read as 0 (adding +0.0 leaves a sum of magnitudes unchanged,
+// so the vector and scalar forms give the same sums).
+__device__ __forceinline__ void load_unit(const float *__restrict__ W, int64_t total, bool vec4, int64_t u,
+                                          float v[4])
 {
-    __shared__ double wsum[kAbsmeanThreads / 32];
-    __shared__ int wbad[kAbsmeanThreads / 32];
-    double s = 0.0;
-    bool bad = false;
-    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
-    // eight loads in flight per thread; the adds keep the plain loop's order
-    for (; i + 7 * stride < total; i += 8 * stride) {
-        float v[8];
+    const int64_t e = 4 * u;
+    if (vec4 && e + 3 < total) {
+        const float4 f = __ldg(reinterpret_cast<const float4 *>(W + e));
+        v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+    } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = W[i + u * stride];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            bad |= !isfinite(v[u]);
-            s += fabs(double(v[u]));
-        }
-    }
-    for (; i < total; i += stride) {
-        const float v = W[i];
-        bad |= !isfinite(v);
-        s += fabs(double(v));
-    }
-    // fixed reduction tree: xor shuffles within the warp, then warps in order
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const bool any_bad = __any_sync(0xffffffffu, bad);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) {
-        wsum[warp] = s;
-        wbad[warp] = any_bad ? 1 : 0;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double t = 0.0;
-        int b = 0;
-        for (int w = 0; w < kAbsmeanThreads / 32; ++w) {
-            t += wsum[w];
-            b |= wbad[w];
-        }
-        scratch->partial[blockIdx.x] = t;
-        scratch->bad[blockIdx.x] = b;
+        for (int i = 0; i < 4; ++i) v[i] = e + i < total ? W[e + i] : 0.f;
     }
 }
 
-__global__ void absmean_scale_kernel(const AbsmeanScratch *scratch, int64_t total, float *scale, int32_t *flags)
+// Block-wide fp64 sum and OR of `bad` by a fixed tree (xor shuffles within
+// each warp, then the warps in order); the result is valid in thread 0.
+__device__ __forceinline__ void block_sum_fixed(double &s, int &bad)
 {
-    if (threadIdx.x != 0) return;
-    double t = 0.0;
-    int b = 0;
-    for (int i = 0; i < kAbsmeanCtas; ++i) {
-        t += scratch->partial[i];
-        b |= scratch->bad[i];
+    __shared__ double wsum[kAbsmeanThreads / 32];
+    __shared__ int wbad[kAbsmeanThreads / 32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    bad = __any_sync(0xffffffffu, bad) ? 1 : 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        wsum[warp] = s;
+        wbad[warp] = bad;
     }
-    if (b) raise_flag(flags, BITNET_FLAG_NONFINITE);
-    *scale = (b || total == 0) ? 0.f : float(t / double(total));
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s = 0.0;
+        bad = 0;
+        for (int w = 0; w < kAbsmeanThreads / 32; ++w) {
+            s += wsum[w];
+            bad |= wbad[w];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kAbsmeanThreads) absmean_partial_kernel(const float *__restrict__ W, int64_t total,
+                                                                       bool vec4, AbsmeanScratch *scratch)
+{
+    const int64_t units = (total + 3) / 4, stride = int64_t(gridDim.x) * blockDim.x;
+    int64_t u = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+    double s = 0.0;
+    int bad = 0;
+    // four units (64 bytes) in flight per thread; the adds keep unit order
+    for (; u + 3 * stride < units; u += 4 * stride) {
+        float v[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) load_unit(W, total, vec4, u + q * stride, v[q]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bad |= !isfinite(v[q][i]);
+                s += fabs(double(v[q][i]));
+            }
+    }
+    for (; u < units; u += stride) {
+        float v[4];
+        load_unit(W, total, vec4, u, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            bad |= !isfinite(v[i]);
+            s += fabs(double(v[i]));
+        }
+    }
+    block_sum_fixed(s, bad);
+    if (threadIdx.x == 0) {
+        scratch->partial[blockIdx.x] = s;
+        scratch->bad[blockIdx.x] = bad;
+    }
 }
 
 // One thread per packed 32-bit word: bytes 4t .. 4t+3 of block j hold, in
 // field g, elements 128j + 32g + 4t + i (i = 0..3) -- four consecutive
 // weights per field, read by 8 consecutive threads as 128 contiguous bytes.
-__global__ void absmean_pack_kernel(const float *__restrict__ W, int64_t n, int64_t k, int64_t kb, bool vec4,
-                                    const float *__restrict__ scale, uint32_t *__restrict__ packed)
+__global__ void __launch_bounds__(kAbsmeanThreads) absmean_pack_kernel(
+    const float *__restrict__ W, int64_t n, int64_t k, int64_t kb, bool vec4, const AbsmeanScratch *scratch,
+    float *scale_out, int32_t *flags, uint32_t *__restrict__ packed)
 {
-    const float s = *scale;
-    const int64_t row_words = 8 * kb, total = n * row_words;
-    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+    __shared__ float s_shared;
+    {
+        double p = 0.0;
+        int bad = 0;
+        for (int i = threadIdx.x; i < kAbsmeanCtas; i += kAbsmeanThreads) {
+            p += scratch->partial[i];
+            bad |= scratch->bad[i];
+        }
+        block_sum_fixed(p, bad);
+        if (threadIdx.x == 0) {
+            const int64_t total = n * k;
+            const float s = bad ? 0.f : float(p / double(total));
+            s_shared = s;
+            if (blockIdx.x == 0) {
+                *scale_out = s;
+                if (bad) raise_flag(flags, BITNET_FLAG_NONFINITE);
+            }
+        }
+        __syncthreads();
+    }
+    const float s = s_shared;
+    const double zero_below = double(s) * kHalfPlusHalfUlp;   // |W| <= this  <=>  code 0
+    const int64_t row_words = 8 * kb, total_words = n * row_words;
+    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total_words;
          idx += int64_t(gridDim.x) * blockDim.x) {
         const int64_t r = idx / row_words, wi = idx - r * row_words;
         const int64_t j = wi >> 3, t = wi & 7;
@@ -231,11 +282,9 @@ __global__ void absmean_pack_kernel(const float *__restrict__ W, int64_t n, int6
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint32_t code = 1;   // weight 0: tails, and every weight when s == 0
-                if (k0 + i < k && s != 0.f) {
-                    const float q = fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -1.f), 1.f);
-                    code = uint32_t(int(q) + 1);
-                }
+                // weight 0 for tails, for every weight when s == 0, and for |W| <= s/2
+                uint32_t code = 1;
+                if (k0 + i < k && s != 0.f && fabs(double(v[i])) > zero_below) code = v[i] > 0.f ? 2u : 0u;
                 out |= code << (8 * i + 2 * g);
             }
         }
@@ -273,16 +322,17 @@ cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float
 }
 
 cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
-                                 int32_t *flags, cudaStream_t st)
+                                 int32_t *flags, int sm_count, cudaStream_t st)
 {
-    const int64_t kb = (k + 127) / 128;
+    const int64_t kb = (k + 127) / 128, words = n * 8 * kb;
     auto *scratch = static_cast<AbsmeanScratch *>(workspace);
-    absmean_partial_kernel<<<kAbsmeanCtas, kAbsmeanThreads, 0, st>>>(w, n * k, scratch);
-    absmean_scale_kernel<<<1, 32, 0, st>>>(scratch, n * k, scale, flags);
-    // float4 loads need every row start 16-byte aligned: W aligned and k % 4 == 0
-    const bool vec4 = (reinterpret_cast<uintptr_t>(w) & 15) == 0 && k % 4 == 0;
-    absmean_pack_kernel<<<grid_for(n * 8 * kb, 256), 256, 0, st>>>(w, n, k, kb, vec4, scale,
-                                                                  reinterpret_cast<uint32_t *>(packed));
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(w) & 15) == 0;
+    absmean_partial_kernel<<<kAbsmeanCtas, kAbsmeanThreads, 0, st>>>(w, n * k, aligned16, scratch);
+    // the pack's float4 loads need every row start 16-byte aligned: W aligned and k % 4 == 0
+    const int64_t want = (words + kAbsmeanThreads - 1) / kAbsmeanThreads;
+    const int grid = int(want < int64_t(kAbsmeanPackCtasPerSm) * sm_count ? want : int64_t(kAbsmeanPackCtasPerSm) * sm_count);
+    absmean_pack_kernel<<<grid, kAbsmeanThreads, 0, st>>>(w, n, k, kb, aligned16 && k % 4 == 0, scratch, scale,
+                                                          flags, reinterpret_cast<uint32_t *>(packed));
     return cudaGetLastError();
 }
 

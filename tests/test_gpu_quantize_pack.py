@@ -82,6 +82,38 @@ def test_quantize_pack_exact_halves_round_to_even():
     assert not back[:, 0::2].any() and (np.abs(back[:, 1::2]) == 1).all()
 
 
+def test_quantize_pack_decisions_next_to_one_half():
+    """Scale exactly 1 (a bulk of +-1/2 and +-3/2 entries; a handful of probes
+    moves the fp64 mean by far less than half an ulp of 1), probes at 1/2 and
+    its neighbouring floats: 1/2 and below give 0, the next float above gives
+    +-1."""
+    n, k = 64, 520
+    mag = np.where(np.arange(n * k).reshape(n, k) % 2 == 0, np.float32(0.5), np.float32(1.5))
+    W = mag.copy()
+    up = np.nextafter(np.float32(0.5), np.float32(1))
+    down = np.nextafter(np.float32(0.5), np.float32(0))
+    probes = [up, -up, down, -down, np.float32(0.5), np.float32(-0.5), np.nextafter(up, np.float32(1))]
+    for i, v in enumerate(probes):
+        W[3, 2 * i] = v
+    packed, s, flags = _run(W)
+    w_or, s_or, _ = oracle.absmean_ternary(W)
+    assert s == np.float32(1.0) == s_or and flags == 0
+    want, _ = oracle.pack(w_or)
+    np.testing.assert_array_equal(packed, want)
+    back = oracle.unpack(packed, k)
+    assert list(back[3, 0:14:2]) == [1, -1, 0, 0, 0, 0, 1]
+
+
+@pytest.mark.parametrize("magnitude", [1e-40, 1e-30, 1e30, 3e37])
+def test_quantize_pack_extreme_magnitudes(magnitude):
+    """Subnormal and very large weights: the scale and every code still match
+    the oracle's fp32 divide (denormals are not flushed on either side)."""
+    rng = np.random.default_rng(int(np.log10(magnitude)) + 100)
+    W = (synth.normal(rng, 37, 333).astype(np.float64) * magnitude).astype(np.float32)
+    assert np.isfinite(W).all()
+    assert _check_against_oracle(W)
+
+
 def test_quantize_pack_all_zero_tensor():
     W = np.zeros((17, 333), np.float32)
     packed, s, flags = _run(W)
