@@ -23,6 +23,7 @@ for _name, _args, _ret in [
     ("oracle_pack", [_P, _i64, _i64, _P], _C.c_int),
     ("oracle_absmean_ternary", [_P, _i64, _i64, _P, _P], _C.c_int),
     ("oracle_ternary_round", [_P, _i64, _f32, _P], None),
+    ("oracle_epilogue", [_P, _P, _P, _C.c_int, _i64, _i64, _P, _P], None),
     ("oracle_unpack", [_P, _i64, _i64, _P], None),
     ("oracle_unpack_misread64", [_P, _i64, _i64, _P], None),
     ("oracle_ternary_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
@@ -140,6 +141,23 @@ def linear(x, packed, n, k, s_w):
     st = _lib.oracle_linear(_ptr(x), m, k, _ptr(packed), n, float(s_w),
                             _ptr(acc), _ptr(y64), _ptr(y32))
     return acc, y64, y32, st
+
+
+def epilogue(y32=None, y64=None, bias=None, gamma=None, residual=None, relu=False):
+    """Fused epilogue (reading R6) on copies of y32 fp32 [m,n] and/or y64 fp64
+    [m,n]: h = relu(y + bias); out = residual + gamma * h.  Returns (y32, y64)."""
+    ref = y32 if y32 is not None else y64
+    m, n = ref.shape
+    y32 = None if y32 is None else _np.array(y32, _np.float32, copy=True, order="C")
+    y64 = None if y64 is None else _np.array(y64, _np.float64, copy=True, order="C")
+    b = None if bias is None else _c(bias, _np.float32)
+    g = None if gamma is None else _c(gamma, _np.float32)
+    r = None if residual is None else _c(residual, _np.float32)
+    assert b is None or b.shape == (n,)
+    assert g is None or g.shape == (n,)
+    assert r is None or r.shape == (m, n)
+    _lib.oracle_epilogue(_ptr(b), _ptr(g), _ptr(r), 1 if relu else 0, m, n, _ptr(y32), _ptr(y64))
+    return y32, y64
 
 
 def linear_rows(x, packed, n, k, s_w, rows):

@@ -203,6 +203,40 @@ int oracle_linear(const float *x, int64_t m, int64_t k, const uint8_t *packed,
     return status;
 }
 
+/* R6 -- the fused epilogue after the dequantisation, in the order of the
+ * technical report's §2.4.1 operator fusion: matrix multiply + bias + ReLU
+ * (mul_mat_add_relu), then residual addition with a layer-scale factor
+ * (add_scaled):  h = relu(y + bias[c]);  out = residual[r,c] + gamma[c] * h.
+ * Each operand is optional (NULL: the step is skipped; relu == 0: no ReLU).
+ * The fp32 form rounds every step once (no fused multiply-add); relu(h) is
+ * h when h > 0 and +0 otherwise.  The fp64 form applies the same steps to
+ * y64 in double precision. */
+void oracle_epilogue(const float *bias, const float *gamma, const float *residual, int relu,
+                     int64_t m, int64_t n, float *y32, double *y64)
+{
+    for (int64_t r = 0; r < m; ++r) {
+        for (int64_t c = 0; c < n; ++c) {
+            const int64_t i = r * n + c;
+            if (y32) {
+                float h = y32[i];
+                if (bias) h = h + bias[c];
+                if (relu) h = h > 0.0f ? h : 0.0f;
+                if (gamma) h = gamma[c] * h;
+                if (residual) h = residual[i] + h;
+                y32[i] = h;
+            }
+            if (y64) {
+                double h = y64[i];
+                if (bias) h = h + (double)bias[c];
+                if (relu) h = h > 0.0 ? h : 0.0;
+                if (gamma) h = (double)gamma[c] * h;
+                if (residual) h = (double)residual[i] + h;
+                y64[i] = h;
+            }
+        }
+    }
+}
+
 int oracle_linear_rows(const float *x, int64_t m, int64_t k, const uint8_t *packed,
                        int64_t n, float s_w, const int64_t *idx, int64_t cnt,
                        int32_t *acc, double *y64)

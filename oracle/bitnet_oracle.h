@@ -94,6 +94,14 @@ void oracle_dequant(const int32_t *acc, const float *s_act, float s_w,
 int oracle_linear(const float *x, int64_t m, int64_t k, const uint8_t *packed,
                   int64_t n, float s_w, int32_t *acc, double *y64, float *y32);
 
+/* R6 -- fused epilogue applied in place to a layer's outputs (fp32 form y32
+ * and/or fp64 form y64, each [m, n]; either may be NULL):
+ *   h = relu(y + bias[c]);  out = residual[r, c] + gamma[c] * h
+ * bias, gamma [n] and residual [m, n] may each be NULL (step skipped);
+ * relu != 0 applies h > 0 ? h : +0. */
+void oracle_epilogue(const float *bias, const float *gamma, const float *residual, int relu,
+                     int64_t m, int64_t n, float *y32, double *y64);
+
 /* Sampled outputs of one layer: only the rows listed in idx[0..cnt) of the
  * weight matrix are computed; acc/y64 are [m, cnt]. */
 int oracle_linear_rows(const float *x, int64_t m, int64_t k, const uint8_t *packed,

@@ -384,3 +384,91 @@ def test_absmean_codes_are_the_second_pass_at_its_own_scale():
     W = (rng.standard_normal((9, 301)) * 0.1).astype(np.float32)
     w, s, _ = oracle.absmean_ternary(W)
     np.testing.assert_array_equal(oracle.ternary_round(W, s), w)
+
+
+# ----------------------------------------------------- fused epilogue (R6)
+
+def _read_epilogue_golden():
+    cases, cur = [], {}
+    for line in open(os.path.join(GOLDEN, "epilogue_small.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, val = (t.strip() for t in line.split(":", 1))
+        if val == "none":
+            cur[key] = None
+        elif key in ("s_w", "relu"):
+            cur[key] = float(val)
+        else:
+            cur[key] = np.array([[float(v) for v in r.split()] for r in val.split("|")], np.float32)
+        if key == "out":
+            cases.append(cur)
+            cur = {}
+    return cases
+
+
+def test_epilogue_golden_examples():
+    cases = _read_epilogue_golden()
+    assert len(cases) == 5
+    for c in cases:
+        w = c["w"].astype(np.int8)
+        n, k = w.shape
+        packed, _ = oracle.pack(w)
+        acc, y64, y32, st = oracle.linear(c["x"], packed, n, k, c["s_w"])
+        assert st == oracle.OK
+        bias = None if c["bias"] is None else c["bias"][0]
+        gamma = None if c["gamma"] is None else c["gamma"][0]
+        o32, o64 = oracle.epilogue(y32, y64, bias=bias, gamma=gamma, residual=c["residual"], relu=bool(c["relu"]))
+        np.testing.assert_array_equal(o32, c["out"])
+        np.testing.assert_array_equal(o64, c["out"].astype(np.float64))
+
+
+def test_epilogue_step_order():
+    """Bias before ReLU, layer scale after ReLU, layer scale not applied to
+    the residual -- each single-element case tells one wrong order apart."""
+    y = np.array([[-1.0]], np.float32)
+    one = np.array([1.0], np.float32)
+    # bias then relu: relu(-1 + 2) = 1  (relu first would give 0 + 2 = 2)
+    assert oracle.epilogue(y, bias=2 * one, relu=True)[0][0, 0] == 1.0
+    # relu then gamma: relu(-1) * -1 = 0  (gamma first would give relu(1) = 1)
+    assert oracle.epilogue(y, gamma=-one, relu=True)[0][0, 0] == 0.0
+    # residual + gamma * h: 1 + 2 * 1 = 3  (gamma * (r + h) would give 4)
+    assert oracle.epilogue(-y, gamma=2 * one, residual=np.array([[1.0]], np.float32))[0][0, 0] == 3.0
+
+
+def test_epilogue_identities_and_exact_cases():
+    rng = np.random.default_rng(61)
+    m, n = 5, 77
+    y = (rng.standard_normal((m, n)) * 3).astype(np.float32)
+    # no operand: bit-for-bit unchanged
+    np.testing.assert_array_equal(oracle.epilogue(y)[0].view(np.uint32), y.view(np.uint32))
+    # residual = -y, nothing else: every x + (-x) is exactly +0
+    out = oracle.epilogue(y, residual=-y)[0]
+    assert (out.view(np.uint32) == 0).all()
+    # power-of-two layer scale scales exactly (no residual)
+    b = rng.standard_normal(n).astype(np.float32)
+    base = oracle.epilogue(y, bias=b, relu=True)[0]
+    four = oracle.epilogue(y, bias=b, relu=True, gamma=np.full(n, 4.0, np.float32))[0]
+    np.testing.assert_array_equal(four, base * np.float32(4))
+    # relu: non-negative, +0 (not -0) wherever y + b <= 0, y + b elsewhere
+    yb = y + b
+    assert (base >= 0).all() and (base.view(np.uint32)[yb <= 0] == 0).all()
+    np.testing.assert_array_equal(base[yb > 0], yb[yb > 0])
+    negzero = np.full((1, 3), -0.0, np.float32)
+    assert (oracle.epilogue(negzero, relu=True)[0].view(np.uint32) == 0).all()
+
+
+def test_epilogue_fp32_form_within_its_rounding_bound_of_fp64_form():
+    """Four rounded fp32 steps: |out32 - out64| <= 4 u (|r| + |g| (|y| + |b|))
+    with u = 2^-24, for inputs exactly representable in both forms."""
+    rng = np.random.default_rng(62)
+    m, n = 7, 301
+    y = (rng.standard_normal((m, n)) * 10).astype(np.float32)
+    b = rng.standard_normal(n).astype(np.float32)
+    g = rng.uniform(0.5, 2.0, n).astype(np.float32)
+    r = (rng.standard_normal((m, n)) * 10).astype(np.float32)
+    o32, o64 = oracle.epilogue(y, y.astype(np.float64), bias=b, gamma=g, residual=r, relu=True)
+    bound = 4 * 2.0 ** -24 * (np.abs(r) + np.abs(g) * (np.abs(y) + np.abs(b))) + 1e-300
+    assert (np.abs(o32.astype(np.float64) - o64) <= bound).all()
+    # and a single dropped term in either form would break it by far
+    assert np.abs(o64 - oracle.epilogue(None, y.astype(np.float64), bias=b, gamma=g, relu=True)[1]).min() > 0
