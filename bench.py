@@ -328,6 +328,37 @@ def run_gpu(args):
             sweep[str(ms)] = {"tokens_per_s": round(whole_job_rate(world, ms, t2 / 50), 1),
                               "weight_gbs": round(stack_bytes / (k2 * 1e-3) / 1e9, 1)}
 
+    # the same M=1 stack with the fused epilogue on every linear: bias, layer
+    # scale and residual add (ReLU on gate and up), residuals in one buffer
+    epi_line = None
+    if m == 1:
+        r_dev = torch.randn(y_dev.numel(), dtype=torch.float32, device=dev)
+        b_dev = torch.randn(y_dev.numel() // m, dtype=torch.float32, device=dev)
+        g_dev = torch.rand(y_dev.numel() // m, dtype=torch.float32, device=dev) + 0.5
+        epis, off = [], 0
+        for i, (y, tw) in enumerate(zip(ys, tws)):
+            n = y.shape[1]
+            name = synth_layer_name(i)
+            epis.append(tw2.make_epilogue(bias=b_dev[off:off + n], gamma=g_dev[off:off + n],
+                                          residual=r_dev[off * m:(off + n) * m].view(m, n),
+                                          relu=name in ("gate", "up")))
+            off += n
+        ce = tw2.StackCall(xs, tws, ys, epis=epis)
+        ce(flags=flags)
+        torch.cuda.synchronize()
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge):
+            ce(flags=flags)
+        te, _ = time_device(ge.replay, 50, 5, stream)
+        te = _max_over_ranks(te) / 50
+        epi_line = {"workload": "the M=1 stack with bias + layer scale + residual add on all %d linears "
+                                "(ReLU on gate/up)" % len(tws),
+                    "tokens_per_s": round(whole_job_rate(world, m, te), 1), "ms_per_step": round(te, 5),
+                    "vs_plain_stack": round(ms_step / te, 4),
+                    "extra_bytes_per_step": int(3 * 4 * y_dev.numel())}
+        if int(flags.item()) != 0:
+            raise RuntimeError(f"device flags {int(flags.item())} in the epilogue stack run")
+
     prefill = None
     if not args.no_prefill:
         prefill = run_prefill(dev, stream, flags, world)
@@ -359,10 +390,16 @@ def run_gpu(args):
             "m_sweep": sweep,
             "prefill": prefill,
             "quantize_pack": qpack,
+            "fused_epilogue_stack": epi_line,
         }
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+def synth_layer_name(i):
+    from ternary_weight_i2_b200 import synth
+    return synth.LAYER_SHAPES[i % len(synth.LAYER_SHAPES)][0]
 
 
 PREFILL_M = 2048
@@ -418,6 +455,24 @@ def run_prefill(dev, stream, flags, world):
     tq, _ = time_device(gq.replay, 20, 3, stream)
     tg, per = time_device(gg.replay, 20, 3, stream)
     tq, tg = _max_over_ranks(tq) / 20, _max_over_ranks(tg) / 20
+    # the same launch with the fused epilogue on every layer (bias, layer
+    # scale, residual add; ReLU on gate and up)
+    epi_keep, epis = [], []
+    for name, n, k, tw in tws:
+        b = torch.randn(n, device=dev)
+        g = torch.rand(n, device=dev) + 0.5
+        r = torch.randn((PREFILL_M, n), device=dev)
+        epi_keep.append((b, g, r))
+        epis.append(tw2.make_epilogue(bias=b, gamma=g, residual=r, relu=name in ("gate", "up")))
+    grouped_epi = tw2.GroupedCall([xq[k] for (_, _, k, _) in tws], [xs_scale[k] for (_, _, k, _) in tws],
+                                  [tw for (_, _, _, tw) in tws], ys, epis=epis)
+    grouped_epi(flags=flags)
+    torch.cuda.synchronize()
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge):
+        grouped_epi(flags=flags)
+    te, _ = time_device(ge.replay, 20, 3, stream)
+    te = _max_over_ranks(te) / 20
     per_shape = {}
     for (name, n, k, tw), y in zip(tws, ys):
         g1 = torch.cuda.CUDAGraph()
@@ -437,6 +492,9 @@ def run_prefill(dev, stream, flags, world):
                          "unit": "TOPS", "frac": round(tops / world / peak, 4),
                          "peak_kind": "measured bf16 cuBLAS burst (MEASURED_PEAKS.json) x 2 (int8:bf16 dense ratio)"},
             "quant_ms_per_step": round(tq, 5), "per_shape": per_shape,
+            "with_fused_epilogue": {"ms_per_step": round(te, 5),
+                                    "tops": round(whole_job_rate(world, PREFILL_OPS, te) / 1e12, 1),
+                                    "epilogue": "bias + layer scale + residual add on all seven (ReLU on gate/up)"},
             "kernel": "gemm_i2_kernel (tcgen05.mma kind::i8, weights expanded into TMEM as A, activations as B from shared memory, 128 features x 192 tokens x 128 tiles, one grouped launch)"}
 
 

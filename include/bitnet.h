@@ -98,6 +98,33 @@ typedef struct {
     float scale;
 } bitnet_tw;
 
+/*
+ * Optional fused epilogue of a linear layer, applied to each output after
+ * the dequantisation y = ((float)acc * s_act[m]) * s_w, in the order of the
+ * technical report's §2.4.1 operator fusion (matrix multiply + bias + ReLU,
+ * then residual addition with a layer-scale factor):
+ *   h   = y + bias[c]                 (bias != NULL)
+ *   h   = h > 0 ? h : +0              (relu != 0)
+ *   h   = gamma[c] * h                (gamma != NULL)
+ *   out = residual[r, c] + h          (residual != NULL)
+ * Every step is one rounded fp32 operation (no fused multiply-add), so the
+ * result equals the oracle's bit for bit.  All pointers are device memory:
+ *   bias, gamma  fp32 [n]
+ *   residual     fp32 [m, n] row-major; it may be the output y itself (an
+ *                in-place residual add: each element is read before it is
+ *                written, by the same thread), but must not overlap any other
+ *                output of the same call.
+ * The int32 accumulators (acc_out) are not affected.  An all-NULL, relu = 0
+ * epilogue is the plain layer.
+ */
+typedef struct {
+    const float *bias;
+    const float *gamma;
+    const float *residual;
+    int32_t relu;
+    int32_t reserved;   /* must be 0 */
+} bitnet_epilogue;
+
 #define BITNET_MAX_K 65536
 /* Largest number of tokens the decode (GEMV) path takes in one pass; larger M
  * runs through the tensor-core GEMM path. */
@@ -252,6 +279,30 @@ BITNET_API bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const 
 BITNET_API bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet_tw *w,
                                   int64_t count, float *const *y, int32_t *const *acc_out,
                                   int32_t *d_flags, void *stream);
+
+/*
+ * The entry points above with a fused epilogue (bitnet_epilogue).  Arguments,
+ * layouts and errors are those of the call without the suffix; `epi` is a
+ * host pointer to one descriptor (bitnet_linear_ex, bitnet_linear_q_ex) or a
+ * host array of `count` descriptors, one per layer (the stack and grouped
+ * calls), and may be NULL (no epilogue).  The residual of layer i is
+ * [m, w[i].n]; m > BITNET_GEMV_MAX_M on the stack call is processed in
+ * slices like the outputs.  A descriptor with reserved != 0 returns
+ * BITNET_ERR_INVALID_ARG.
+ */
+BITNET_API bitnet_status bitnet_linear_ex(const float *x, int64_t m, const bitnet_tw *w, const bitnet_epilogue *epi,
+                                          float *y, int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                                          int32_t *d_flags, void *stream);
+BITNET_API bitnet_status bitnet_linear_q_ex(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
+                                            const bitnet_epilogue *epi, float *y, int32_t *acc_out,
+                                            int32_t *d_flags, void *stream);
+BITNET_API bitnet_status bitnet_linear_q_grouped_ex(const int8_t *const *xq, const float *const *act_scale,
+                                                    int64_t m, const bitnet_tw *w, const bitnet_epilogue *epi,
+                                                    int64_t count, float *const *y, int32_t *const *acc_out,
+                                                    int32_t *d_flags, void *stream);
+BITNET_API bitnet_status bitnet_linear_stack_ex(const float *const *x, int64_t m, const bitnet_tw *w,
+                                                const bitnet_epilogue *epi, int64_t count, float *const *y,
+                                                int32_t *const *acc_out, int32_t *d_flags, void *stream);
 
 /*
  * bitnet_linear_stack with no device allocation, for callers that cannot call

@@ -5,7 +5,7 @@ The compute lives in ``libbitnet.so`` (CUDA kernels behind the C ABI of
 used by callers for device memory and streams.
 """
 from ._abi import (  # noqa: F401
-    BitnetError, StackCall, TW, header_functions, kpad, linear, linear_q, linear_stack,
+    BitnetError, Epilogue, StackCall, TW, make_epilogue, header_functions, kpad, linear, linear_q, linear_stack,
     linear_stack_noalloc, linear_q_grouped, GroupedCall,
     linear_workspace_bytes, load, make_tw, pack_ternary, packed_bytes, quant_act,
     quantize_pack, quantize_pack_workspace_bytes,

@@ -28,6 +28,13 @@ class TW(C.Structure):
     _fields_ = [("packed", C.c_void_p), ("n", C.c_int64), ("k", C.c_int64), ("scale", C.c_float)]
 
 
+class Epilogue(C.Structure):
+    """bitnet_epilogue: fused bias / ReLU / layer-scaled residual add (device
+    pointers, NULL = step skipped)."""
+    _fields_ = [("bias", C.c_void_p), ("gamma", C.c_void_p), ("residual", C.c_void_p),
+                ("relu", C.c_int32), ("reserved", C.c_int32)]
+
+
 class BitnetError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -53,6 +60,11 @@ _SIGNATURES = {
     "bitnet_linear_stack": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_linear_q_grouped": ([_P, _P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_linear_stack_noalloc": ([_P, _I64, C.POINTER(TW), _I64, _P, _P, _P, _P], C.c_int),
+    "bitnet_linear_ex": ([_P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
+    "bitnet_linear_q_ex": ([_P, _P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _P, _P, _P, _P], C.c_int),
+    "bitnet_linear_q_grouped_ex": ([_P, _P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _I64, _P, _P, _P, _P],
+                                   C.c_int),
+    "bitnet_linear_stack_ex": ([_P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _I64, _P, _P, _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
     "bitnet_debug_set_trace": ([_P], C.c_int),
@@ -184,23 +196,37 @@ def make_tw(packed, n: int, k: int, scale: float) -> TW:
     return TW(packed.data_ptr(), n, k, float(scale))
 
 
-def linear(x, tw: TW, y, acc=None, workspace=None, flags=None, stream=None) -> None:
+def make_epilogue(bias=None, gamma=None, residual=None, relu=False) -> Epilogue:
+    """Epilogue descriptor from optional device tensors: bias [n], gamma [n],
+    residual [m, n] (may be the output tensor itself)."""
+    return Epilogue(_ptr(bias), _ptr(gamma), _ptr(residual), 1 if relu else 0, 0)
+
+
+def linear(x, tw: TW, y, acc=None, workspace=None, flags=None, stream=None, epi: Epilogue | None = None) -> None:
     m = x.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load().bitnet_linear(_ptr(x), m, C.byref(tw), _ptr(y), _ptr(acc), _ptr(workspace),
-                                ws_bytes, _ptr(flags), _stream(stream)), "bitnet_linear")
+    if epi is None:
+        _check(load().bitnet_linear(_ptr(x), m, C.byref(tw), _ptr(y), _ptr(acc), _ptr(workspace),
+                                    ws_bytes, _ptr(flags), _stream(stream)), "bitnet_linear")
+    else:
+        _check(load().bitnet_linear_ex(_ptr(x), m, C.byref(tw), C.byref(epi), _ptr(y), _ptr(acc), _ptr(workspace),
+                                       ws_bytes, _ptr(flags), _stream(stream)), "bitnet_linear_ex")
 
 
-def linear_q(xq, act_scale, tw: TW, y, acc=None, flags=None, stream=None) -> None:
+def linear_q(xq, act_scale, tw: TW, y, acc=None, flags=None, stream=None, epi: Epilogue | None = None) -> None:
     m = xq.shape[0]
-    _check(load().bitnet_linear_q(_ptr(xq), _ptr(act_scale), m, C.byref(tw), _ptr(y), _ptr(acc),
-                                  _ptr(flags), _stream(stream)), "bitnet_linear_q")
+    if epi is None:
+        _check(load().bitnet_linear_q(_ptr(xq), _ptr(act_scale), m, C.byref(tw), _ptr(y), _ptr(acc),
+                                      _ptr(flags), _stream(stream)), "bitnet_linear_q")
+    else:
+        _check(load().bitnet_linear_q_ex(_ptr(xq), _ptr(act_scale), m, C.byref(tw), C.byref(epi), _ptr(y),
+                                         _ptr(acc), _ptr(flags), _stream(stream)), "bitnet_linear_q_ex")
 
 
 class GroupedCall:
     """Marshalled arguments of one bitnet_linear_q_grouped call (reusable)."""
 
-    def __init__(self, xqs, scales, tws, ys, accs=None):
+    def __init__(self, xqs, scales, tws, ys, accs=None, epis=None):
         count = len(tws)
         self.count = count
         self.m = xqs[0].shape[0]
@@ -211,23 +237,30 @@ class GroupedCall:
         self.acc_arr = None
         if accs is not None:
             self.acc_arr = (C.c_void_p * count)(*[(a.data_ptr() if a is not None else None) for a in accs])
+        self.epi_arr = None if epis is None else (Epilogue * count)(*[e if e is not None else Epilogue()
+                                                                      for e in epis])
         self._keep = (xqs, scales, ys, accs)
 
     def __call__(self, flags=None, stream=None) -> None:
-        _check(load().bitnet_linear_q_grouped(self.xq_arr, self.s_arr, self.m, self.tw_arr, self.count,
-                                              self.y_arr, self.acc_arr, _ptr(flags), _stream(stream)),
-               "bitnet_linear_q_grouped")
+        if self.epi_arr is None:
+            _check(load().bitnet_linear_q_grouped(self.xq_arr, self.s_arr, self.m, self.tw_arr, self.count,
+                                                  self.y_arr, self.acc_arr, _ptr(flags), _stream(stream)),
+                   "bitnet_linear_q_grouped")
+        else:
+            _check(load().bitnet_linear_q_grouped_ex(self.xq_arr, self.s_arr, self.m, self.tw_arr, self.epi_arr,
+                                                     self.count, self.y_arr, self.acc_arr, _ptr(flags),
+                                                     _stream(stream)), "bitnet_linear_q_grouped_ex")
 
 
-def linear_q_grouped(xqs, scales, tws, ys, accs=None, flags=None, stream=None) -> None:
-    GroupedCall(xqs, scales, tws, ys, accs)(flags=flags, stream=stream)
+def linear_q_grouped(xqs, scales, tws, ys, accs=None, flags=None, stream=None, epis=None) -> None:
+    GroupedCall(xqs, scales, tws, ys, accs, epis)(flags=flags, stream=stream)
 
 
 class StackCall:
     """Marshalled arguments of one bitnet_linear_stack call, built once and
     reusable (the pointer arrays are kept alive by this object)."""
 
-    def __init__(self, xs, tws, ys, accs=None):
+    def __init__(self, xs, tws, ys, accs=None, epis=None):
         count = len(tws)
         self.count = count
         self.m = xs[0].shape[0]
@@ -237,16 +270,23 @@ class StackCall:
         self.acc_arr = None
         if accs is not None:
             self.acc_arr = (C.c_void_p * count)(*[(a.data_ptr() if a is not None else None) for a in accs])
+        self.epi_arr = None if epis is None else (Epilogue * count)(*[e if e is not None else Epilogue()
+                                                                      for e in epis])
         self._keep = (xs, ys, accs)
 
     def __call__(self, flags=None, stream=None) -> None:
-        _check(load().bitnet_linear_stack(self.x_arr, self.m, self.tw_arr, self.count, self.y_arr,
-                                          self.acc_arr, _ptr(flags), _stream(stream)),
-               "bitnet_linear_stack")
+        if self.epi_arr is None:
+            _check(load().bitnet_linear_stack(self.x_arr, self.m, self.tw_arr, self.count, self.y_arr,
+                                              self.acc_arr, _ptr(flags), _stream(stream)),
+                   "bitnet_linear_stack")
+        else:
+            _check(load().bitnet_linear_stack_ex(self.x_arr, self.m, self.tw_arr, self.epi_arr, self.count,
+                                                 self.y_arr, self.acc_arr, _ptr(flags), _stream(stream)),
+                   "bitnet_linear_stack_ex")
 
 
-def linear_stack(xs, tws, ys, accs=None, flags=None, stream=None) -> None:
-    StackCall(xs, tws, ys, accs)(flags=flags, stream=stream)
+def linear_stack(xs, tws, ys, accs=None, flags=None, stream=None, epis=None) -> None:
+    StackCall(xs, tws, ys, accs, epis)(flags=flags, stream=stream)
 
 
 def linear_stack_noalloc(xs, tws, ys, accs=None, flags=None, stream=None) -> None:

@@ -23,13 +23,13 @@ cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float
 cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
                                  int32_t *flags, int sm_count, cudaStream_t st);
 bool gemm_available();
-cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count,
-                        uint64_t *trace, cudaStream_t st);
+cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
+                        const bitnet_epilogue *epi, float *y, int32_t *acc, int32_t *flags, uint64_t wait_limit,
+                        int force_stall, int sm_count, uint64_t *trace, cudaStream_t st);
 cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
-                                const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
-                                int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count, uint64_t *trace,
-                                cudaStream_t st);
+                                const bitnet_tw *w, const bitnet_epilogue *epi, int count, float *const *y,
+                                int32_t *const *acc, int32_t *flags, uint64_t wait_limit, int force_stall,
+                                int sm_count, uint64_t *trace, cudaStream_t st);
 }  // namespace bitnet
 
 using namespace bitnet;
@@ -107,6 +107,16 @@ bitnet_status check_tw(const bitnet_tw &w, int64_t i)
     if (w.k < 1 || w.k > BITNET_MAX_K)
         return fail(BITNET_ERR_INVALID_ARG, "layer %lld: k=%lld out of range [1, %d]", (long long)i, (long long)w.k,
                     BITNET_MAX_K);
+    return BITNET_OK;
+}
+
+// A fused-epilogue descriptor (may be NULL: no epilogue).
+bitnet_status check_epi(const bitnet_epilogue *e, int64_t i)
+{
+    if (!e) return BITNET_OK;
+    if (e->reserved != 0) return fail(BITNET_ERR_INVALID_ARG, "layer %lld: epilogue reserved field not 0", (long long)i);
+    if (!aligned(e->bias, 4) || !aligned(e->gamma, 4) || !aligned(e->residual, 4))
+        return fail(BITNET_ERR_INVALID_ARG, "layer %lld: epilogue operand not 4-byte aligned", (long long)i);
     return BITNET_OK;
 }
 
@@ -227,6 +237,10 @@ struct LayerReq {
     bitnet_tw w;
     float *y;
     int32_t *acc;
+    const float *bias;     // fused epilogue operands (null when absent)
+    const float *gamma;
+    const float *res;      // this slice's residual rows
+    int64_t relu;
 };
 
 // Kernel variant for m tokens whose activation area holds an input of
@@ -338,8 +352,15 @@ bitnet_status plan_and_launch(const std::vector<LayerReq> &L, int m, bool prequa
         p.lin[i].n = int32_t(L[i].w.n);
         p.lin[i].kb = int32_t(blocks_of(L[i].w.k));
         p.lin[i].scale = L[i].w.scale;
-        p.lin[i].input = found;
+        p.lin[i].input = int16_t(found);
+        p.lin[i].bias = L[i].bias;
+        p.lin[i].gamma = L[i].gamma;
+        p.lin[i].res = L[i].res;
+        p.lin[i].relu = L[i].relu ? 1 : 0;
     }
+    p.has_epi = 0;
+    for (int i = 0; i < count; ++i)
+        if (L[i].bias || L[i].gamma || L[i].res || L[i].relu) p.has_epi = 1;
     const int variant = pick_variant(m, max_kpad);
     if (variant < 0)
         return fail(BITNET_ERR_INVALID_ARG, "m=%d x kpad=%lld exceeds the GEMV activation area", m,
@@ -591,11 +612,12 @@ size_t bitnet_linear_workspace_bytes(int64_t m, int64_t k)
 }
 
 static bitnet_status gemv_slices(const float *const *x, const int8_t *const *xq, const float *const *xs, int64_t m,
-                                 const bitnet_tw *w, int64_t count, float *const *y, int32_t *const *acc,
-                                 int32_t *d_flags, cudaStream_t st, const DevInfo &dev)
+                                 const bitnet_tw *w, const bitnet_epilogue *epi, int64_t count, float *const *y,
+                                 int32_t *const *acc, int32_t *d_flags, cudaStream_t st, const DevInfo &dev)
 {
     std::vector<LayerReq> L;
     L.resize(static_cast<size_t>(count));
+    std::memset(static_cast<void *>(L.data()), 0, L.size() * sizeof(LayerReq));   // plan keys compare bytes
     for (int64_t m0 = 0; m0 < m; m0 += BITNET_GEMV_MAX_M) {
         const int ms = int((m - m0) < BITNET_GEMV_MAX_M ? (m - m0) : BITNET_GEMV_MAX_M);
         for (int64_t i = 0; i < count; ++i) {
@@ -610,6 +632,10 @@ static bitnet_status gemv_slices(const float *const *x, const int8_t *const *xq,
             L[i].w = w[i];
             L[i].y = y[i] + m0 * w[i].n;
             L[i].acc = (acc && acc[i]) ? acc[i] + m0 * w[i].n : nullptr;
+            L[i].bias = epi ? epi[i].bias : nullptr;
+            L[i].gamma = epi ? epi[i].gamma : nullptr;
+            L[i].res = (epi && epi[i].residual) ? epi[i].residual + m0 * w[i].n : nullptr;
+            L[i].relu = (epi && epi[i].relu) ? 1 : 0;
         }
         bitnet_status s = plan_and_launch(L, ms, xq != nullptr, d_flags, st, dev);
         if (s != BITNET_OK) return s;
@@ -617,12 +643,15 @@ static bitnet_status gemv_slices(const float *const *x, const int8_t *const *xq,
     return BITNET_OK;
 }
 
-bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_tw *w, float *y, int32_t *acc_out,
-                            void *workspace, size_t workspace_bytes, int32_t *d_flags, void *stream)
+bitnet_status bitnet_linear_ex(const float *x, int64_t m, const bitnet_tw *w, const bitnet_epilogue *epi, float *y,
+                               int32_t *acc_out, void *workspace, size_t workspace_bytes, int32_t *d_flags,
+                               void *stream)
 {
     if (!x || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "linear: NULL pointer");
     if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "linear: bad m=%lld", (long long)m);
     bitnet_status s = check_tw(*w, 0);
+    if (s != BITNET_OK) return s;
+    s = check_epi(epi, 0);
     if (s != BITNET_OK) return s;
     if (!aligned(x, 16)) return fail(BITNET_ERR_INVALID_ARG, "linear: x not 16-byte aligned");
     const size_t need = bitnet_linear_workspace_bytes(m, w->k);
@@ -645,28 +674,37 @@ bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_tw *w, float
             const float *xsa[1] = {xs};
             float *ya[1] = {y};
             int32_t *aa[1] = {acc_out};
-            return gemv_slices(nullptr, xqa, xsa, m, w, 1, ya, aa, d_flags, st, dev);
+            return gemv_slices(nullptr, xqa, xsa, m, w, epi, 1, ya, aa, d_flags, st, dev);
         }
         const float *xa[1] = {x};
         float *ya[1] = {y};
         int32_t *aa[1] = {acc_out};
-        return gemv_slices(xa, nullptr, nullptr, m, w, 1, ya, aa, d_flags, st, dev);
+        return gemv_slices(xa, nullptr, nullptr, m, w, epi, 1, ya, aa, d_flags, st, dev);
     }
     int8_t *xq = static_cast<int8_t *>(workspace);
     const size_t qa = (size_t(m) * size_t(128 * blocks_of(w->k)) + 255) / 256 * 256;
     float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + qa);
     cudaError_t e = launch_quant(x, m, w->k, xq, xs, d_flags, st);
     if (e != cudaSuccess) return cuda_fail(e, "quant launch");
-    e = launch_gemm(xq, xs, m, w, y, acc_out, d_flags, wait_limit(), g_force_stall, dev.sm_count, g_trace, st);
+    e = launch_gemm(xq, xs, m, w, epi, y, acc_out, d_flags, wait_limit(), g_force_stall, dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 
-bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                              int32_t *acc_out, int32_t *d_flags, void *stream)
+bitnet_status bitnet_linear(const float *x, int64_t m, const bitnet_tw *w, float *y, int32_t *acc_out,
+                            void *workspace, size_t workspace_bytes, int32_t *d_flags, void *stream)
+{
+    return bitnet_linear_ex(x, m, w, nullptr, y, acc_out, workspace, workspace_bytes, d_flags, stream);
+}
+
+bitnet_status bitnet_linear_q_ex(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
+                                 const bitnet_epilogue *epi, float *y, int32_t *acc_out, int32_t *d_flags,
+                                 void *stream)
 {
     if (!xq || !act_scale || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "linear_q: NULL pointer");
     if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "linear_q: bad m");
     bitnet_status s = check_tw(*w, 0);
+    if (s != BITNET_OK) return s;
+    s = check_epi(epi, 0);
     if (s != BITNET_OK) return s;
     if (!aligned(xq, 16)) return fail(BITNET_ERR_INVALID_ARG, "linear_q: xq not 16-byte aligned");
     DevInfo dev;
@@ -678,15 +716,22 @@ bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t 
         const float *xsa[1] = {act_scale};
         float *ya[1] = {y};
         int32_t *aa[1] = {acc_out};
-        return gemv_slices(nullptr, xqa, xsa, m, w, 1, ya, aa, d_flags, st, dev);
+        return gemv_slices(nullptr, xqa, xsa, m, w, epi, 1, ya, aa, d_flags, st, dev);
     }
-    cudaError_t e = launch_gemm(xq, act_scale, m, w, y, acc_out, d_flags, wait_limit(), g_force_stall, dev.sm_count, g_trace, st);
+    cudaError_t e = launch_gemm(xq, act_scale, m, w, epi, y, acc_out, d_flags, wait_limit(), g_force_stall,
+                                dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "gemm launch");
 }
 
-bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
-                                      const bitnet_tw *w, int64_t count, float *const *y, int32_t *const *acc_out,
-                                      int32_t *d_flags, void *stream)
+bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
+                              int32_t *acc_out, int32_t *d_flags, void *stream)
+{
+    return bitnet_linear_q_ex(xq, act_scale, m, w, nullptr, y, acc_out, d_flags, stream);
+}
+
+bitnet_status bitnet_linear_q_grouped_ex(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                         const bitnet_tw *w, const bitnet_epilogue *epi, int64_t count,
+                                         float *const *y, int32_t *const *acc_out, int32_t *d_flags, void *stream)
 {
     if (!xq || !act_scale || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: NULL array");
     if (count < 1 || count > BITNET_GROUP_MAX)
@@ -701,20 +746,32 @@ bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *cons
         if (!aligned(xq[i], 16) || !aligned(y[i], 16))
             return fail(BITNET_ERR_INVALID_ARG, "linear_q_grouped: layer %lld xq or y not 16-byte aligned",
                         (long long)i);
+        if (epi) {
+            s = check_epi(epi + i, i);
+            if (s != BITNET_OK) return s;
+        }
     }
     DevInfo dev;
     bitnet_status s = check_device(&dev);
     if (s != BITNET_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (m <= BITNET_GEMV_MAX_M)
-        return gemv_slices(nullptr, xq, act_scale, m, w, count, y, acc_out, d_flags, st, dev);
-    cudaError_t e = launch_gemm_grouped(xq, act_scale, m, w, int(count), y, acc_out, d_flags, wait_limit(),
+        return gemv_slices(nullptr, xq, act_scale, m, w, epi, count, y, acc_out, d_flags, st, dev);
+    cudaError_t e = launch_gemm_grouped(xq, act_scale, m, w, epi, int(count), y, acc_out, d_flags, wait_limit(),
                                         g_force_stall, dev.sm_count, g_trace, st);
     return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "grouped gemm launch");
 }
 
-bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet_tw *w, int64_t count,
-                                  float *const *y, int32_t *const *acc_out, int32_t *d_flags, void *stream)
+bitnet_status bitnet_linear_q_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
+                                      const bitnet_tw *w, int64_t count, float *const *y, int32_t *const *acc_out,
+                                      int32_t *d_flags, void *stream)
+{
+    return bitnet_linear_q_grouped_ex(xq, act_scale, m, w, nullptr, count, y, acc_out, d_flags, stream);
+}
+
+bitnet_status bitnet_linear_stack_ex(const float *const *x, int64_t m, const bitnet_tw *w, const bitnet_epilogue *epi,
+                                     int64_t count, float *const *y, int32_t *const *acc_out, int32_t *d_flags,
+                                     void *stream)
 {
     if (!x || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "stack: NULL array");
     if (count < 1 || count > BITNET_STACK_MAX)
@@ -726,11 +783,22 @@ bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet
         if (s != BITNET_OK) return s;
         if (!x[i] || !y[i]) return fail(BITNET_ERR_INVALID_ARG, "stack: layer %lld has a NULL x or y", (long long)i);
         if (!aligned(x[i], 16)) return fail(BITNET_ERR_INVALID_ARG, "stack: layer %lld x not 16-byte aligned", (long long)i);
+        if (epi) {
+            bitnet_status s = check_epi(epi + i, i);
+            if (s != BITNET_OK) return s;
+        }
     }
     DevInfo dev;
     bitnet_status s = check_device(&dev);
     if (s != BITNET_OK) return s;
-    return gemv_slices(x, nullptr, nullptr, m, w, count, y, acc_out, d_flags, static_cast<cudaStream_t>(stream), dev);
+    return gemv_slices(x, nullptr, nullptr, m, w, epi, count, y, acc_out, d_flags, static_cast<cudaStream_t>(stream),
+                       dev);
+}
+
+bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet_tw *w, int64_t count,
+                                  float *const *y, int32_t *const *acc_out, int32_t *d_flags, void *stream)
+{
+    return bitnet_linear_stack_ex(x, m, w, nullptr, count, y, acc_out, d_flags, stream);
 }
 
 }  // extern "C"
@@ -810,8 +878,13 @@ bitnet_status noalloc_plan_and_launch(int count, int m, int32_t *flags, cudaStre
         p.lin[i].n = int32_t(L[i].w.n);
         p.lin[i].kb = int32_t(blocks_of(L[i].w.k));
         p.lin[i].scale = L[i].w.scale;
-        p.lin[i].input = found;
+        p.lin[i].input = int16_t(found);
+        p.lin[i].bias = nullptr;
+        p.lin[i].gamma = nullptr;
+        p.lin[i].res = nullptr;
+        p.lin[i].relu = 0;
     }
+    p.has_epi = 0;
     const int variant = pick_variant(m, max_kpad);
     if (variant < 0)
         return fail(BITNET_ERR_INVALID_ARG, "noalloc stack: m=%d x kpad=%lld exceeds the GEMV activation area", m,
@@ -962,6 +1035,8 @@ extern "C" bitnet_status bitnet_linear_stack_noalloc(const float *const *x, int6
             r.w = w[i];
             r.y = y[i] + m0 * w[i].n;
             r.acc = (acc_out && acc_out[i]) ? acc_out[i] + m0 * w[i].n : nullptr;
+            r.bias = r.gamma = r.res = nullptr;
+            r.relu = 0;
         }
         s = noalloc_plan_and_launch(n, ms, d_flags, st, dev, maps);
         if (s != BITNET_OK) return s;

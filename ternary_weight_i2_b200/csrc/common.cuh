@@ -38,6 +38,15 @@ __device__ __forceinline__ void raise_flag(int32_t *flags, int32_t bit)
     if (flags) atomicOr(flags, bit);
 }
 
+// 4-byte asynchronous copy global -> shared (no registers held while in
+// flight), committed as a group and waited for by the issuing thread.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)

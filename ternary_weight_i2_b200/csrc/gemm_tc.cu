@@ -78,6 +78,10 @@ struct GemmProblem {
     const float *act_scale;   // [M]
     float *y;                 // [M, N]
     int32_t *acc;             // [M, N] or null
+    const float *bias;        // fused epilogue: [N] or null
+    const float *gamma;       // [N] or null (layer scale)
+    const float *res;         // [M, N] or null (residual; may be y)
+    int32_t relu;             // ReLU after the bias
     float w_scale;
     int32_t m, n, kb;
     int32_t tiles_t, tiles_f;
@@ -95,6 +99,7 @@ struct GemmParams {
     int32_t *flags;
     uint64_t wait_limit;
     int32_t force_stall;      // test aid: K block kStallBlock's copies are never issued
+    int32_t has_epi;          // some problem of the launch has a fused-epilogue operand
     uint64_t *trace;          // optional: CTA 0 stamps (kGemmTraceMisc + 72 entries)
     int32_t cta_off[kMaxGemmCtas + 1];   // CTA c runs tiles[cta_off[c] .. cta_off[c+1])
     int32_t tiles[kMaxGemmTiles];        // tile ids, heaviest first within each CTA
@@ -291,6 +296,9 @@ __device__ __forceinline__ int tile_tokens(const GemmProblem &P, int t_tile)
     return min(kBT, P.m - t_tile * kBT);
 }
 
+// kEpi: the launch has a fused-epilogue operand on some problem.  The plain
+// instantiation carries none of the epilogue code.
+template <bool kEpi>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_constant__ GemmParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -509,18 +517,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
             int32_t *const acc = P.acc;
             const float *const act_scale = P.act_scale;
             const float sw = P.w_scale;
+            const float *const res = kEpi ? P.res : nullptr;
+            const bool has_bias = kEpi && P.bias != nullptr, has_gamma = kEpi && P.gamma != nullptr;
+            const bool relu = kEpi && P.relu != 0;
+            const float *const bias_p = P.bias, *const gamma_p = P.gamma;
             const int b = tcount & 1, ur = tcount >> 1;
             // the tile's activation scales, token 32c + lane in sa_t[c], fetched
             // while the accumulator is still being computed
             float sa_t[kBT / 32];
 #pragma unroll
             for (int c = 0; c < kBT / 32; ++c) sa_t[c] = (32 * c + lane < nt) ? act_scale[t0 + 32 * c + lane] : 0.f;
+            const int f = tr.f_tile * kBF + 32 * quad + lane;
+            const bool f_ok = f < n;
+            // fused epilogue operands of this thread's feature (technical
+            // report §2.4.1: bias + ReLU, then the layer-scaled residual add)
+            const float bias_f = (has_bias && f_ok) ? bias_p[f] : 0.f;
+            const float gamma_f = (has_gamma && f_ok) ? gamma_p[f] : 1.f;
+            const bool has_res = res != nullptr && f_ok;
             bool live = warp_wait_progress(smem_u32(&accf_bar[b]), ur & 1, long_limit);
             if (!live && lane == 0) fail();
             live = __shfl_sync(0xffffffffu, (live && *abort_flag == 0) ? 1 : 0, 0) != 0;
             tc_fence_after();
-            const int f = tr.f_tile * kBF + 32 * quad + lane;
-            const bool f_ok = f < n;
             const uint32_t taddr = tmem_base + lane_addr + uint32_t(b * kBT);
             if (live) {
 #pragma unroll
@@ -550,6 +567,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_i2_kernel(const __grid_c
                     for (int j = 0; j < 32; ++j)
                         v[j] = __float_as_uint(
                             __fmul_rn(__fmul_rn(float(int32_t(v[j])), __shfl_sync(0xffffffffu, sa_l, j)), sw));
+                    // each step one rounding, in straight-line loops (the
+                    // branches are uniform over the tile)
+                    if (has_bias) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__fadd_rn(__uint_as_float(v[j]), bias_f));
+                    }
+                    if (relu) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(v[j]) > 0.f ? v[j] : 0u;
+                    }
+                    if (has_gamma) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__fmul_rn(gamma_f, __uint_as_float(v[j])));
+                    }
+                    if (has_res) {
+                        const float *rc = res + size_t(t0 + c0) * size_t(n) + f;
+                        if (full) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                v[j] = __float_as_uint(__fadd_rn(rc[size_t(j) * size_t(n)], __uint_as_float(v[j])));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (c0 + j < nt)
+                                    v[j] = __float_as_uint(__fadd_rn(rc[size_t(j) * size_t(n)], __uint_as_float(v[j])));
+                        }
+                    }
                     if (f_ok) {
                         float *yc = y + size_t(t0 + c0) * size_t(n) + f;
                         if (full) {
@@ -605,7 +649,8 @@ bool gemm_available() { return true; }
 // (cost = MMA work of the tile's K loop plus a fixed epilogue share), so
 // layers of different K balance inside one persistent launch.
 cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act_scale, int64_t m,
-                                const bitnet_tw *w, int count, float *const *y, int32_t *const *acc,
+                                const bitnet_tw *w, const bitnet_epilogue *epi, int count, float *const *y,
+                                int32_t *const *acc,
                                 int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count, uint64_t *trace,
                                 cudaStream_t st)
 {
@@ -645,6 +690,10 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
         P.act_scale = act_scale[g];
         P.y = y[g];
         P.acc = acc ? acc[g] : nullptr;
+        P.bias = epi ? epi[g].bias : nullptr;
+        P.gamma = epi ? epi[g].gamma : nullptr;
+        P.res = epi ? epi[g].residual : nullptr;
+        P.relu = (epi && epi[g].relu) ? 1 : 0;
         P.w_scale = w[g].scale;
         P.m = int32_t(m);
         P.n = int32_t(w[g].n);
@@ -666,13 +715,19 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
     p.wait_limit = wait_limit;
     p.force_stall = force_stall;
     p.trace = trace;
+    p.has_epi = 0;
+    for (int g = 0; g < count; ++g)
+        if (p.prob[g].bias || p.prob[g].gamma || p.prob[g].res || p.prob[g].relu) p.has_epi = 1;
     std::stable_sort(all.begin(), all.end(), [](const Tile &a, const Tile &b) { return a.cost > b.cost; });
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     static bool configured[64] = {};
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_i2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+        cudaError_t e = cudaFuncSetAttribute(gemm_i2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kGemmSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gemm_i2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -700,23 +755,26 @@ cudaError_t launch_gemm_grouped(const int8_t *const *xq, const float *const *act
             const int c = owner[i];
             p.tiles[p.cta_off[c] + fill[c]++] = all[c0 + i].id;
         }
-        gemm_i2_kernel<<<G, kGemmThreads, kGemmSmem, st>>>(p);
+        if (p.has_epi)
+            gemm_i2_kernel<true><<<G, kGemmThreads, kGemmSmem, st>>>(p);
+        else
+            gemm_i2_kernel<false><<<G, kGemmThreads, kGemmSmem, st>>>(p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
-cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w, float *y,
-                        int32_t *acc, int32_t *flags, uint64_t wait_limit, int force_stall, int sm_count,
-                        uint64_t *trace, cudaStream_t st)
+cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
+                        const bitnet_epilogue *epi, float *y, int32_t *acc, int32_t *flags, uint64_t wait_limit,
+                        int force_stall, int sm_count, uint64_t *trace, cudaStream_t st)
 {
     const int8_t *xqa[1] = {xq};
     const float *sa[1] = {act_scale};
     float *ya[1] = {y};
     int32_t *aa[1] = {acc};
-    return launch_gemm_grouped(xqa, sa, m, w, 1, ya, acc ? aa : nullptr, flags, wait_limit, force_stall, sm_count,
-                               trace, st);
+    return launch_gemm_grouped(xqa, sa, m, w, epi, 1, ya, acc ? aa : nullptr, flags, wait_limit, force_stall,
+                               sm_count, trace, st);
 }
 
 }  // namespace bitnet

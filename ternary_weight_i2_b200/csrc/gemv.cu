@@ -50,6 +50,7 @@ struct SegInfo {
     int32_t slot;    // range-local input slot
     int32_t tile0;   // first tile of the layer in this range
     int32_t tcum;    // range-local index of the segment's first tile
+    int32_t lin;     // index of the layer in the launch (its epilogue operands)
     float scale;
 };
 
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
             si.slot = sg.slot;
             si.tile0 = sg.tile0;
             si.scale = L.scale;
+            si.lin = sg.lin;
             cnt = sg.tile1 - sg.tile0;
         }
         int incl = cnt;
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
         if (jj < nblk) block_dot<M>(wrow, rx, xb, kp, jj, acc0);
         if (cc == si.nch - 1) {
             const int row = (si.tile0 + (ci - si.tcum)) * kTileRows + lane;
-            if (row < si.n) {
+            if (row < si.n && !p.has_epi) {
 #pragma unroll
                 for (int m = 0; m < M; ++m) {
                     const int32_t s64 = (acc0[m][0] + acc1[m][0]) * 64 + (acc0[m][1] + acc1[m][1]) * 16 +
@@ -400,6 +402,29 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_stack_kernel(const __grid_con
                     const float yv = __fmul_rn(__fmul_rn(float(a), meta->s_act[u * M + m]), si.scale);
                     si.y[size_t(m) * size_t(si.n) + row] = yv;
                     if (si.acc) si.acc[size_t(m) * size_t(si.n) + row] = a;
+                }
+            } else if (row < si.n) {
+                // fused epilogue operands (technical report §2.4.1): bias and
+                // ReLU, then the layer-scaled residual add; one rounding per step
+                const GemvLinear &L = p.lin[si.lin];
+                const float *res = L.res;
+                const bool relu = L.relu != 0;
+                const float bias = L.bias ? __ldg(L.bias + row) : 0.f;
+                const float gamma = L.gamma ? __ldg(L.gamma + row) : 1.f;
+                const bool has_bias = L.bias != nullptr, has_gamma = L.gamma != nullptr;
+#pragma unroll
+                for (int m = 0; m < M; ++m) {
+                    const int32_t s64 = (acc0[m][0] + acc1[m][0]) * 64 + (acc0[m][1] + acc1[m][1]) * 16 +
+                                        (acc0[m][2] + acc1[m][2]) * 4 + (acc0[m][3] + acc1[m][3]);
+                    const int32_t a = (s64 >> 6) - meta->sumx[u * M + m];
+                    float yv = __fmul_rn(__fmul_rn(float(a), meta->s_act[u * M + m]), si.scale);
+                    if (has_bias) yv = __fadd_rn(yv, bias);
+                    if (relu) yv = yv > 0.f ? yv : 0.f;
+                    if (has_gamma) yv = __fmul_rn(gamma, yv);
+                    const size_t o = size_t(m) * size_t(si.n) + row;
+                    if (res) yv = __fadd_rn(res[o], yv);
+                    si.y[o] = yv;
+                    if (si.acc) si.acc[o] = a;
                 }
             }
 #pragma unroll

@@ -44,10 +44,14 @@ struct GemvLinear {
     const void *tmap;        // device CUtensorMap of packed [n, 32*kb] bytes, box 128 x 32
     float *y;                // [m, n]
     int32_t *acc;            // [m, n] or null
+    const float *bias;       // fused epilogue: [n] or null
+    const float *gamma;      // [n] or null (layer scale)
+    const float *res;        // [m, n] or null (residual; may be y)
     int32_t n;
     int32_t kb;              // 128-element blocks per row
     float scale;             // s_w
-    int32_t input;           // index into inputs[]
+    int16_t input;           // index into inputs[]
+    int16_t relu;            // fused epilogue: ReLU after the bias
 };
 
 struct GemvInput {
@@ -78,6 +82,7 @@ struct GemvParams {
     uint64_t wait_limit;
     int32_t x_bytes;         // bytes of the shared-memory activation area
     int32_t fence_maps;      // tensor maps may have been rewritten at a reused address
+    int32_t has_epi;         // some layer of the launch has a fused-epilogue operand
     uint64_t *trace;         // optional: kTraceEvents globaltimer stamps per warp
     GemvLinear lin[kMaxLinears];
     GemvInput inp[kMaxInputs];
