@@ -109,11 +109,12 @@ typedef struct {
  *   out = residual[r, c] + h          (residual != NULL)
  * Every step is one rounded fp32 operation (no fused multiply-add), so the
  * result equals the oracle's bit for bit.  All pointers are device memory:
- *   bias, gamma  fp32 [n]
- *   residual     fp32 [m, n] row-major; it may be the output y itself (an
- *                in-place residual add: each element is read before it is
- *                written, by the same thread), but must not overlap any other
- *                output of the same call.
+ *   bias, gamma  fp32 [n], 4-byte aligned; must not overlap any output of
+ *                the call (they are read through the read-only cache)
+ *   residual     fp32 [m, n] row-major, 4-byte aligned; it may be the output
+ *                y itself (an in-place residual add: each element is read
+ *                before it is written, by the same thread), but must not
+ *                overlap any other output of the same call.
  * The int32 accumulators (acc_out) are not affected.  An all-NULL, relu = 0
  * epilogue is the plain layer.
  */

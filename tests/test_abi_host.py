@@ -103,3 +103,62 @@ def test_library_refuses_missing_build(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         _abi.load(str(tmp_path / "missing.so"))
+
+
+def test_quantize_pack_rejects_bad_arguments_before_any_device_call(lib):
+    P = C.c_void_p
+    good = P(0x10000)
+    ws_bytes = lib.bitnet_quantize_pack_workspace_bytes()
+    assert ws_bytes == tw2.quantize_pack_workspace_bytes() >= 1024 * 12
+
+    def call(w=good, n=4, k=4, packed=good, scale=good, ws=good, wsb=ws_bytes):
+        return lib.bitnet_quantize_pack(w, n, k, packed, scale, ws, wsb, None, None)
+
+    assert call(w=None) == _abi.ERR_INVALID_ARG
+    assert call(scale=None) == _abi.ERR_INVALID_ARG
+    assert call(ws=None) == _abi.ERR_INVALID_ARG
+    assert call(n=0) == _abi.ERR_INVALID_ARG
+    assert call(k=65537) == _abi.ERR_INVALID_ARG
+    assert call(w=P(0x10002)) == _abi.ERR_INVALID_ARG          # fp32 input not 4-byte aligned
+    assert call(packed=P(0x10004)) == _abi.ERR_INVALID_ARG     # packed rows need 16 bytes
+    assert call(ws=P(0x10004)) == _abi.ERR_INVALID_ARG         # fp64 partials need 8 bytes
+    assert call(wsb=ws_bytes - 1) == _abi.ERR_WORKSPACE
+    assert b"workspace" in lib.bitnet_last_error()
+
+
+def test_epilogue_descriptor_checked_before_any_device_call(lib):
+    """A reserved field other than 0 or a misaligned operand is refused on
+    every entry point that takes an epilogue, before the device is touched."""
+    P = C.c_void_p
+    good = P(0x10000)
+    w = _tw()
+    bad_reserved = _abi.Epilogue(None, None, None, 0, 1)
+    bad_align = _abi.Epilogue(0x10002, None, None, 0, 0)
+    for epi in (bad_reserved, bad_align):
+        assert lib.bitnet_linear_ex(good, 1, C.byref(w), C.byref(epi), good, None, None, 0, None, None) \
+            == _abi.ERR_INVALID_ARG
+        assert lib.bitnet_linear_q_ex(good, good, 1, C.byref(w), C.byref(epi), good, None, None, None) \
+            == _abi.ERR_INVALID_ARG
+        xs = (C.c_void_p * 2)(0x10000, 0x10000)
+        ys = (C.c_void_p * 2)(0x20000, 0x30000)
+        ws = (_abi.TW * 2)(_tw(), _tw())
+        epis = (_abi.Epilogue * 2)(_abi.Epilogue(), epi)   # the second layer's is bad
+        assert lib.bitnet_linear_stack_ex(xs, 1, ws, epis, 2, ys, None, None, None) == _abi.ERR_INVALID_ARG
+        assert b"layer 1" in lib.bitnet_last_error()
+        assert lib.bitnet_linear_q_grouped_ex(xs, xs, 16, ws, epis, 2, ys, None, None, None) \
+            == _abi.ERR_INVALID_ARG
+    assert C.sizeof(_abi.Epilogue) == 32   # three pointers and two int32 (bitnet_epilogue)
+
+
+@pytest.mark.skipif(_has_gpu(), reason="checks the no-device path")
+def test_epilogue_forms_report_no_device(lib):
+    """Well-formed epilogue calls on a machine without a usable CUDA device
+    fail with a device error rather than succeeding silently."""
+    P = C.c_void_p
+    w = _tw()
+    epi = _abi.Epilogue(0x40000, 0x50000, 0x60000, 1, 0)
+    st = lib.bitnet_linear_ex(P(0x10000), 1, C.byref(w), C.byref(epi), P(0x20000), None, None, 0, None, None)
+    assert st in (_abi.ERR_CUDA, _abi.ERR_UNSUPPORTED_DEVICE)
+    st = lib.bitnet_quantize_pack(P(0x10000), 4, 4, P(0x20000), P(0x30000), P(0x40000),
+                                  lib.bitnet_quantize_pack_workspace_bytes(), None, None)
+    assert st in (_abi.ERR_CUDA, _abi.ERR_UNSUPPORTED_DEVICE)
