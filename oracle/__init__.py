@@ -24,6 +24,9 @@ for _name, _args, _ret in [
     ("oracle_absmean_ternary", [_P, _i64, _i64, _P, _P], _C.c_int),
     ("oracle_ternary_round", [_P, _i64, _f32, _P], None),
     ("oracle_epilogue", [_P, _P, _P, _C.c_int, _i64, _i64, _P, _P], None),
+    ("oracle_i8_row_bytes", [_i64], _i64),
+    ("oracle_i8_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
+    ("oracle_linear_i8", [_P, _i64, _i64, _P, _i64, _f32, _P, _P, _P], _C.c_int),
     ("oracle_unpack", [_P, _i64, _i64, _P], None),
     ("oracle_unpack_misread64", [_P, _i64, _i64, _P], None),
     ("oracle_ternary_matmul", [_P, _i64, _P, _i64, _i64, _P], _C.c_int),
@@ -158,6 +161,42 @@ def epilogue(y32=None, y64=None, bias=None, gamma=None, residual=None, relu=Fals
     assert r is None or r.shape == (m, n)
     _lib.oracle_epilogue(_ptr(b), _ptr(g), _ptr(r), 1 if relu else 0, m, n, _ptr(y32), _ptr(y64))
     return y32, y64
+
+
+def i8_row_bytes(k: int) -> int:
+    return int(_lib.oracle_i8_row_bytes(k))
+
+
+def i8_layout(w):
+    """int8 weights [n,k] -> the I8_S row layout [n, 32*ceil(k/32)], pads 0
+    (reading R7)."""
+    w = _c(w, _np.int8)
+    n, k = w.shape
+    out = _np.zeros((n, i8_row_bytes(k)), _np.int8)
+    out[:, :k] = w
+    return out
+
+
+def i8_matmul(q, w_rows, k):
+    """q int8 [m, kpad] x I8_S rows [n, 32*ceil(k/32)] -> (acc int32 [m,n], status)."""
+    q = _c(q, _np.int8)
+    w_rows = _c(w_rows, _np.int8)
+    m, n = q.shape[0], w_rows.shape[0]
+    acc = _np.empty((m, n), _np.int32)
+    st = _lib.oracle_i8_matmul(_ptr(q), m, _ptr(w_rows), n, k, _ptr(acc))
+    return acc, st
+
+
+def linear_i8(x, w_rows, k, s_w):
+    """I8_S layer (reading R7) -> (acc int32, y64 fp64, y32 fp32, status)."""
+    x = _c(x, _np.float32)
+    w_rows = _c(w_rows, _np.int8)
+    m, n = x.shape[0], w_rows.shape[0]
+    acc = _np.empty((m, n), _np.int32)
+    y64 = _np.empty((m, n), _np.float64)
+    y32 = _np.empty((m, n), _np.float32)
+    st = _lib.oracle_linear_i8(_ptr(x), m, k, _ptr(w_rows), n, float(s_w), _ptr(acc), _ptr(y64), _ptr(y32))
+    return acc, y64, y32, st
 
 
 def linear_rows(x, packed, n, k, s_w, rows):

@@ -203,6 +203,42 @@ int oracle_linear(const float *x, int64_t m, int64_t k, const uint8_t *packed,
     return status;
 }
 
+/* R7 -- I8_S: whole Q_K = 32 blocks per weight row. */
+int64_t oracle_i8_row_bytes(int64_t k) { return 32 * ((k + 31) / 32); }
+
+/* R7, integer part -- the plain int8 x int8 dot product over k < K, summed
+ * in int64 and checked against the int32 range. */
+int oracle_i8_matmul(const int8_t *q, int64_t m, const int8_t *w, int64_t n, int64_t k, int32_t *acc)
+{
+    int status = ORACLE_OK;
+    const int64_t kpad = oracle_kpad(k), rowb = oracle_i8_row_bytes(k);
+    for (int64_t r = 0; r < m; ++r)
+        for (int64_t c = 0; c < n; ++c) {
+            int64_t s = 0;
+            for (int64_t i = 0; i < k; ++i) s += (int64_t)q[r * kpad + i] * (int64_t)w[c * rowb + i];
+            if (s > INT32_MAX) { s = INT32_MAX; status |= ORACLE_OVERFLOW; }
+            if (s < INT32_MIN) { s = INT32_MIN; status |= ORACLE_OVERFLOW; }
+            acc[r * n + c] = (int32_t)s;
+        }
+    return status;
+}
+
+int oracle_linear_i8(const float *x, int64_t m, int64_t k, const int8_t *w, int64_t n, float s_w,
+                     int32_t *acc, double *y64, float *y32)
+{
+    const int64_t kpad = oracle_kpad(k);
+    int8_t *q = (int8_t *)malloc((size_t)(m * kpad));
+    float *sa = (float *)malloc((size_t)m * sizeof(float));
+    int32_t *a = acc ? acc : (int32_t *)malloc((size_t)(m * n) * sizeof(int32_t));
+    int status = oracle_quant_act(x, m, k, q, sa);
+    status |= oracle_i8_matmul(q, m, w, n, k, a);
+    oracle_dequant(a, sa, s_w, m, n, y64, y32);
+    if (!acc) free(a);
+    free(q);
+    free(sa);
+    return status;
+}
+
 /* R6 -- the fused epilogue after the dequantisation, in the order of the
  * technical report's §2.4.1 operator fusion: matrix multiply + bias + ReLU
  * (mul_mat_add_relu), then residual addition with a layer-scale factor

@@ -36,6 +36,18 @@
  *       scale), -1, 1) with the division and the rounding in fp32 (rounding
  *       half to even).  An all-zero tensor gives scale 0 and w = 0; a tensor
  *       holding NaN/Inf gives scale 0, w = 0 and ORACLE_NONFINITE.
+ *  R6 fused epilogue (§2.4.1 operator fusion: multiply + bias + ReLU, then
+ *       residual addition with a layer scale): h = relu(y + bias);
+ *       out = residual + gamma * h; one fp32 rounding per step.
+ *  R7 I8_S linear (§2.2.1 full-pipeline INT8; §2.4.2: the I8_S kernel works
+ *       on blocks of Q_K = 32 elements and shares the maddubs multiply-add
+ *       pipeline with I2_S, using the sign trick for signed x signed):
+ *       weights are plain int8 [N, K] with one fp32 scale per tensor, each
+ *       row stored in 32*ceil(K/32) bytes (whole Q_K blocks, pads 0);
+ *       activations as R1; acc[m,n] = sum_{k<K} q[m,k]*w[n,k], exact integer
+ *       (the sign trick |w| * (sign(w) x) gives the same products);
+ *       y = acc * s_act * s_w as in R4, where (float)acc now rounds to
+ *       nearest even when |acc| > 2^24.
  */
 #ifndef BITNET_ORACLE_H
 #define BITNET_ORACLE_H
@@ -55,6 +67,19 @@ extern "C" {
 /* ceil(K/128) and the padded width 128*ceil(K/128) */
 int64_t oracle_blocks(int64_t k);
 int64_t oracle_kpad(int64_t k);
+
+/* R7: bytes of one I8_S weight row, 32*ceil(K/32) */
+int64_t oracle_i8_row_bytes(int64_t k);
+
+/* R7, integer part: acc [m,n] from quantised q [m, kpad] (R1 layout) and
+ * int8 weights w [n, oracle_i8_row_bytes(k)]; only k < K is read.
+ * Returns ORACLE_OVERFLOW if a sum leaves the int32 range. */
+int oracle_i8_matmul(const int8_t *q, int64_t m, const int8_t *w, int64_t n, int64_t k, int32_t *acc);
+
+/* R7, whole layer: quantise x (R1), contract with the int8 weights, and
+ * dequantise (R4's two forms); acc may be NULL. */
+int oracle_linear_i8(const float *x, int64_t m, int64_t k, const int8_t *w, int64_t n, float s_w,
+                     int32_t *acc, double *y64, float *y32);
 
 /* R1: x fp32 [m,k] -> q int8 [m, kpad] (pads zero), s_act fp32 [m].
  * Returns ORACLE_NONFINITE if any row was non-finite. */

@@ -472,3 +472,82 @@ def test_epilogue_fp32_form_within_its_rounding_bound_of_fp64_form():
     assert (np.abs(o32.astype(np.float64) - o64) <= bound).all()
     # and a single dropped term in either form would break it by far
     assert np.abs(o64 - oracle.epilogue(None, y.astype(np.float64), bias=b, gamma=g, relu=True)[1]).min() > 0
+
+
+# --------------------------------------------------------- I8_S linear (R7)
+
+def _maddubs_dot(q_row, w_row):
+    """The pages' I8_S multiply-add pipeline for one dot product, block by
+    block (Q_K = 32): sign trick (unsigned |w| times sign(w)*x), adjacent
+    products summed into int16 with saturation, int16 pairs into int32, then
+    a horizontal sum.  Written from the pipeline's description, independent
+    of the oracle's plain loop."""
+    k = len(q_row)
+    total = 0
+    for b0 in range(0, k, 32):
+        wb = w_row[b0:b0 + 32].astype(np.int64)
+        xb = q_row[b0:b0 + 32].astype(np.int64)
+        u = np.abs(wb)                                   # u8 operand
+        s = np.sign(wb) * xb                             # s8 operand
+        assert (u <= 255).all() and (s >= -128).all() and (s <= 127).all()
+        prod = u * s
+        if len(prod) % 2:
+            prod = np.append(prod, 0)
+        pairs = np.clip(prod[0::2] + prod[1::2], -32768, 32767)   # maddubs: saturating int16
+        total += int(pairs.sum())                        # madd with ones + hsum in int32
+    return total
+
+
+def test_i8_matmul_brute_force_and_sign_trick_pipeline():
+    rng = np.random.default_rng(71)
+    for m, n, k in [(1, 1, 1), (3, 5, 31), (2, 7, 32), (4, 3, 33), (2, 9, 100), (5, 4, 1536)]:
+        x = synth.normal_outliers(rng, m, k)
+        q, s_act, _ = oracle.quant_act(x)
+        w = rng.integers(-127, 128, size=(n, k), dtype=np.int64).astype(np.int8)
+        acc, st = oracle.i8_matmul(q, oracle.i8_layout(w), k)
+        assert st == oracle.OK
+        want = q[:, :k].astype(np.int64) @ w.astype(np.int64).T
+        np.testing.assert_array_equal(acc, want)
+        for r in range(m):
+            for c in range(n):
+                assert _maddubs_dot(q[r, :k], w[c]) == acc[r, c]
+
+
+def test_i8_matmul_closed_forms_pads_and_overflow():
+    k = 1000
+    q = np.zeros((2, oracle.kpad(k)), np.int8)
+    q[0, :k] = 127
+    q[1, :k] = np.where(np.arange(k) % 2 == 0, 127, -127)
+    w = np.full((3, k), 127, np.int8)
+    w[1] = -127
+    w[2] = np.where(np.arange(k) % 2 == 0, 1, -1)
+    rows = oracle.i8_layout(w)
+    acc, _ = oracle.i8_matmul(q, rows, k)
+    np.testing.assert_array_equal(acc, [[127 * 127 * k, -127 * 127 * k, 0],
+                                        [0, 0, 127 * k]])
+    # pads (k..1023 of each row) are never read
+    rows2 = rows.copy()
+    rows2[:, k:] = 99
+    np.testing.assert_array_equal(oracle.i8_matmul(q, rows2, k)[0], acc)
+    assert oracle.i8_row_bytes(k) == 1024 and oracle.i8_row_bytes(1) == 32 and oracle.i8_row_bytes(32) == 32
+    # past 2^31 / 127^2 = 133,143 elements a saturated sum leaves int32
+    kb = 133200
+    qb = np.full((1, oracle.kpad(kb)), 127, np.int8)
+    wb = np.full((1, kb), 127, np.int8)
+    _, st = oracle.i8_matmul(qb, oracle.i8_layout(wb), kb)
+    assert st & oracle.OVERFLOW
+
+
+def test_linear_i8_fp32_form_rounds_large_sums_to_even():
+    """x = 127 everywhere gives q = 127 and s_act = 1; with w = 127 and
+    s_w = 1, y32 is (float)acc.  K = 1041: acc = 16129 * 1041 = 16,790,289,
+    odd and above 2^24, halfway between 16,790,288 and 16,790,290: rounds to
+    the even 16,790,288."""
+    k = 1041
+    x = np.full((1, k), 127.0, np.float32)
+    w = np.full((1, k), 127, np.int8)
+    acc, y64, y32, st = oracle.linear_i8(x, oracle.i8_layout(w), k, 1.0)
+    assert st == oracle.OK
+    assert acc[0, 0] == 16790289
+    assert y64[0, 0] == 16790289.0
+    assert y32[0, 0] == np.float32(16790288.0)
