@@ -50,6 +50,8 @@ def _args():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the M=2048 prefill GEMM line")
+    ap.add_argument("--i8-only", action="store_true",
+                    help="run only the I8_S decode measurement and print its object")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the M=2048 prefill GEMMs (profiling aid) and print their object")
     ap.add_argument("--soak", type=float, default=0.5,
@@ -363,6 +365,7 @@ def run_gpu(args):
     if not args.no_prefill:
         prefill = run_prefill(dev, stream, flags, world)
     qpack = run_quantize_pack(dev, stream, flags, world)
+    i8_line = run_i8_decode(dev, stream, flags, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -391,6 +394,7 @@ def run_gpu(args):
             "prefill": prefill,
             "quantize_pack": qpack,
             "fused_epilogue_stack": epi_line,
+            "i8s_decode": i8_line,
         }
         print(json.dumps(line))
     if world > 1:
@@ -544,6 +548,56 @@ def run_quantize_pack(dev, stream, flags, world):
             "kernels": "absmean_partial_kernel, absmean_pack_kernel"}
 
 
+I8_LAYERS = 4
+
+
+def run_i8_decode(dev, stream, flags, world):
+    """I8_S decode: M=1 token through four decoder layers' seven linears with
+    int8 weights (one bitnet_linear_i8 call each, 28 per step, graph-replayed;
+    187 MB of weights, larger than L2).  Algorithmic bytes: 1 B per weight."""
+    import torch
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import synth
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.seed_for(6, 0))
+    calls, keep, weight_bytes = [], [], 0
+    xs = {k: torch.randn((1, k), generator=g, device=dev) for k in synth.LAYER_INPUT_K}
+    for L in range(I8_LAYERS):
+        for name, n, k in synth.LAYER_SHAPES:
+            rows = torch.randint(-127, 128, (n, tw2.i8_row_bytes(k)), generator=g, device=dev, dtype=torch.int8)
+            y = torch.empty((1, n), device=dev)
+            ws = torch.empty(tw2.linear_i8_workspace_bytes(1, k), dtype=torch.uint8, device=dev)
+            w8 = tw2.make_i8w(rows, n, k, 0.01)
+            keep.append((rows, y, ws))
+            calls.append((xs[k], w8, y, ws))
+            weight_bytes += n * k
+
+    def step():
+        for x, w8, y, ws in calls:
+            tw2.linear_i8(x, w8, y, ws, flags=flags)
+
+    step()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        step()
+    steps = 20
+    t, _ = time_device(gr.replay, steps, 3, stream)
+    t = _max_over_ranks(t) / steps
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"device flags {int(flags.item())} in the I8_S run")
+    hbm, _, _ = _peaks()
+    gbs = weight_bytes / (t * 1e-3) / 1e9
+    return {"workload": "I8_S decode, M=1, %d decoder layers x seven linears with int8 weights (%.1f MB > L2)"
+                        % (I8_LAYERS, weight_bytes / 1e6),
+            "tokens_per_s": round(whole_job_rate(world, 1, t), 1), "ms_per_step": round(t, 5),
+            "launches_per_step": 2 * len(calls),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes_per_weight": 1.0},
+            "kernels": "quant_kernel + i8_gemv_kernel<1> per linear"}
+
+
 def build_stack_views(m, dev, tws, layers=28):
     """Inputs/outputs for another token count, reusing the packed weights."""
     import torch
@@ -633,7 +687,7 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
-    elif args.prefill_only:
+    elif args.prefill_only or args.i8_only:
         import torch
         import ternary_weight_i2_b200 as tw2
         from ternary_weight_i2_b200 import build as tbuild
@@ -642,7 +696,8 @@ def main():
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         flags = torch.zeros(1, dtype=torch.int32, device=dev)
-        print(json.dumps(run_prefill(dev, torch.cuda.current_stream(), flags, 1)))
+        run = run_prefill if args.prefill_only else run_i8_decode
+        print(json.dumps(run(dev, torch.cuda.current_stream(), flags, 1)))
     else:
         run_gpu(args)
 

@@ -306,6 +306,41 @@ BITNET_API bitnet_status bitnet_linear_stack_ex(const float *const *x, int64_t m
                                                 int32_t *const *acc_out, int32_t *d_flags, void *stream);
 
 /*
+ * I8_S linear layer: int8 weights x per-token int8 activations (technical
+ * report §2.2.1: the full-pipeline INT8 scheme of the VAE tokenizer; §2.4.2:
+ * the I8_S kernel works on blocks of Q_K = 32 elements through the same
+ * multiply-add pipeline as I2_S).  Weights are plain int8 with one fp32
+ * scale per tensor, each row stored as whole Q_K blocks:
+ *   w->w      device int8 [n, bitnet_i8_row_bytes(k)], 16-byte aligned; the
+ *             pad bytes of each row may hold anything (they meet zero
+ *             activations)
+ *   w->scale  s_w
+ * acc[m,n] = sum_{k<K} q[m,k] * w[n,k] exactly; y = ((float)acc * s_act) *
+ * s_w (the int-to-float conversion rounds to nearest even once |acc| > 2^24),
+ * then the optional epilogue (NULL: none).  x, y, acc_out and d_flags as in
+ * bitnet_linear.  The activations are quantised into the caller's workspace
+ * (>= bitnet_linear_i8_workspace_bytes(m, k), 256-byte aligned), then the
+ * GEMV streams the weight rows in slices of at most 8 tokens.
+ */
+typedef struct {
+    const int8_t *w;
+    int64_t n;
+    int64_t k;
+    float scale;
+} bitnet_i8w;
+
+/* Bytes of one I8_S weight row: 32 * ceil(k/32); 0 on bad k. */
+BITNET_API size_t bitnet_i8_row_bytes(int64_t k);
+
+/* Workspace of bitnet_linear_i8: int8 activations [m, bitnet_kpad(k)] and
+ * their scales; 0 on bad sizes. */
+BITNET_API size_t bitnet_linear_i8_workspace_bytes(int64_t m, int64_t k);
+
+BITNET_API bitnet_status bitnet_linear_i8(const float *x, int64_t m, const bitnet_i8w *w, const bitnet_epilogue *epi,
+                                          float *y, int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                                          int32_t *d_flags, void *stream);
+
+/*
  * bitnet_linear_stack with no device allocation, for callers that cannot call
  * cudaMalloc: code running where the allocator is owned by someone else (a
  * host framework with its own pooling allocator, a real-time loop that must not

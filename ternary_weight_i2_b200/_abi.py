@@ -28,6 +28,11 @@ class TW(C.Structure):
     _fields_ = [("packed", C.c_void_p), ("n", C.c_int64), ("k", C.c_int64), ("scale", C.c_float)]
 
 
+class I8W(C.Structure):
+    """bitnet_i8w: one I8_S int8 weight tensor (device pointer + shape + scale)."""
+    _fields_ = [("w", C.c_void_p), ("n", C.c_int64), ("k", C.c_int64), ("scale", C.c_float)]
+
+
 class Epilogue(C.Structure):
     """bitnet_epilogue: fused bias / ReLU / layer-scaled residual add (device
     pointers, NULL = step skipped)."""
@@ -65,6 +70,9 @@ _SIGNATURES = {
     "bitnet_linear_q_grouped_ex": ([_P, _P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _I64, _P, _P, _P, _P],
                                    C.c_int),
     "bitnet_linear_stack_ex": ([_P, _I64, C.POINTER(TW), C.POINTER(Epilogue), _I64, _P, _P, _P, _P], C.c_int),
+    "bitnet_i8_row_bytes": ([_I64], C.c_size_t),
+    "bitnet_linear_i8_workspace_bytes": ([_I64, _I64], C.c_size_t),
+    "bitnet_linear_i8": ([_P, _I64, C.POINTER(I8W), C.POINTER(Epilogue), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
     "bitnet_debug_set_trace": ([_P], C.c_int),
@@ -211,6 +219,28 @@ def linear(x, tw: TW, y, acc=None, workspace=None, flags=None, stream=None, epi:
     else:
         _check(load().bitnet_linear_ex(_ptr(x), m, C.byref(tw), C.byref(epi), _ptr(y), _ptr(acc), _ptr(workspace),
                                        ws_bytes, _ptr(flags), _stream(stream)), "bitnet_linear_ex")
+
+
+def i8_row_bytes(k: int) -> int:
+    return int(load().bitnet_i8_row_bytes(k))
+
+
+def linear_i8_workspace_bytes(m: int, k: int) -> int:
+    return int(load().bitnet_linear_i8_workspace_bytes(m, k))
+
+
+def make_i8w(w_rows, n: int, k: int, scale: float) -> I8W:
+    """I8_S weight descriptor over a device int8 tensor [n, i8_row_bytes(k)]."""
+    return I8W(w_rows.data_ptr(), n, k, float(scale))
+
+
+def linear_i8(x, w8: I8W, y, workspace, acc=None, flags=None, stream=None, epi: Epilogue | None = None) -> None:
+    """I8_S layer: int8 weights x per-token int8 activations (bitnet_linear_i8)."""
+    m = x.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().bitnet_linear_i8(_ptr(x), m, C.byref(w8), None if epi is None else C.byref(epi), _ptr(y),
+                                   _ptr(acc), _ptr(workspace), ws_bytes, _ptr(flags), _stream(stream)),
+           "bitnet_linear_i8")
 
 
 def linear_q(xq, act_scale, tw: TW, y, acc=None, flags=None, stream=None, epi: Epilogue | None = None) -> None:

@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libbitnet.so")
 BUILD_DIR = os.path.join(HERE, "_build")
 
-SOURCES = ["capi.cu", "gemv.cu", "pack_quant.cu", "gemm_tc.cu"]
+SOURCES = ["capi.cu", "gemv.cu", "pack_quant.cu", "gemm_tc.cu", "gemv_i8.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -23,6 +23,9 @@ cudaError_t launch_quant(const float *x, int64_t m, int64_t k, int8_t *xq, float
 cudaError_t launch_quantize_pack(const float *w, int64_t n, int64_t k, uint8_t *packed, float *scale, void *workspace,
                                  int32_t *flags, int sm_count, cudaStream_t st);
 bool gemm_available();
+cudaError_t launch_gemv_i8(const int8_t *w, int64_t n, int64_t k, float s_w, const int8_t *q, const float *s_act,
+                           int64_t m, const bitnet_epilogue *e, float *y, int32_t *acc, int sm_count,
+                           cudaStream_t st);
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
                         const bitnet_epilogue *epi, float *y, int32_t *acc, int32_t *flags, uint64_t wait_limit,
                         int force_stall, int sm_count, uint64_t *trace, cudaStream_t st);
@@ -799,6 +802,48 @@ bitnet_status bitnet_linear_stack(const float *const *x, int64_t m, const bitnet
                                   float *const *y, int32_t *const *acc_out, int32_t *d_flags, void *stream)
 {
     return bitnet_linear_stack_ex(x, m, w, nullptr, count, y, acc_out, d_flags, stream);
+}
+
+size_t bitnet_i8_row_bytes(int64_t k)
+{
+    if (k < 1 || k > BITNET_MAX_K) return 0;
+    return size_t(32 * ((k + 31) / 32));
+}
+
+size_t bitnet_linear_i8_workspace_bytes(int64_t m, int64_t k)
+{
+    if (m < 1 || m > (int64_t(1) << 31) - 1 || k < 1 || k > BITNET_MAX_K) return 0;
+    const size_t a = size_t(m) * size_t(128 * blocks_of(k));
+    return (a + 255) / 256 * 256 + size_t(m) * sizeof(float);
+}
+
+bitnet_status bitnet_linear_i8(const float *x, int64_t m, const bitnet_i8w *w, const bitnet_epilogue *epi, float *y,
+                               int32_t *acc_out, void *workspace, size_t workspace_bytes, int32_t *d_flags,
+                               void *stream)
+{
+    if (!x || !w || !y || !w->w) return fail(BITNET_ERR_INVALID_ARG, "linear_i8: NULL pointer");
+    if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "linear_i8: bad m=%lld", (long long)m);
+    if (w->n < 1 || w->n > (int64_t(1) << 30) || w->k < 1 || w->k > BITNET_MAX_K)
+        return fail(BITNET_ERR_INVALID_ARG, "linear_i8: bad sizes n=%lld k=%lld", (long long)w->n, (long long)w->k);
+    if (!aligned(w->w, 16) || !aligned(x, 16))
+        return fail(BITNET_ERR_INVALID_ARG, "linear_i8: weights or x not 16-byte aligned");
+    bitnet_status s = check_epi(epi, 0);
+    if (s != BITNET_OK) return s;
+    const size_t need = bitnet_linear_i8_workspace_bytes(m, w->k);
+    if (!workspace || workspace_bytes < need)
+        return fail(BITNET_ERR_WORKSPACE, "linear_i8: workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(BITNET_ERR_INVALID_ARG, "linear_i8: workspace not 256-byte aligned");
+    DevInfo dev;
+    s = check_device(&dev);
+    if (s != BITNET_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int8_t *xq = static_cast<int8_t *>(workspace);
+    const size_t qa = (size_t(m) * size_t(128 * blocks_of(w->k)) + 255) / 256 * 256;
+    float *xs = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + qa);
+    cudaError_t e = launch_quant(x, m, w->k, xq, xs, d_flags, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quant launch");
+    e = launch_gemv_i8(w->w, w->n, w->k, w->scale, xq, xs, m, epi, y, acc_out, dev.sm_count, st);
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "i8 gemv launch");
 }
 
 }  // extern "C"
