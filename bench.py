@@ -553,29 +553,30 @@ I8_LAYERS = 4
 
 def run_i8_decode(dev, stream, flags, world):
     """I8_S decode: M=1 token through four decoder layers' seven linears with
-    int8 weights (one bitnet_linear_i8 call each, 28 per step, graph-replayed;
-    187 MB of weights, larger than L2).  Algorithmic bytes: 1 B per weight."""
+    int8 weights, all 28 in one bitnet_linear_i8_grouped call per step
+    (graph-replayed; 187 MB of weights, larger than L2).  Algorithmic bytes:
+    1 B per weight."""
     import torch
     import ternary_weight_i2_b200 as tw2
     from ternary_weight_i2_b200 import synth
 
     g = torch.Generator(device=dev)
     g.manual_seed(synth.seed_for(6, 0))
-    calls, keep, weight_bytes = [], [], 0
+    keep, xs_l, w8s, ys, weight_bytes = [], [], [], [], 0
     xs = {k: torch.randn((1, k), generator=g, device=dev) for k in synth.LAYER_INPUT_K}
     for L in range(I8_LAYERS):
         for name, n, k in synth.LAYER_SHAPES:
             rows = torch.randint(-127, 128, (n, tw2.i8_row_bytes(k)), generator=g, device=dev, dtype=torch.int8)
-            y = torch.empty((1, n), device=dev)
-            ws = torch.empty(tw2.linear_i8_workspace_bytes(1, k), dtype=torch.uint8, device=dev)
-            w8 = tw2.make_i8w(rows, n, k, 0.01)
-            keep.append((rows, y, ws))
-            calls.append((xs[k], w8, y, ws))
+            keep.append(rows)
+            w8s.append(tw2.make_i8w(rows, n, k, 0.01))
+            xs_l.append(xs[k])
+            ys.append(torch.empty((1, n), device=dev))
             weight_bytes += n * k
+    call = tw2.I8GroupCall(xs_l, w8s, ys)
+    ws = torch.empty(call.workspace_bytes, dtype=torch.uint8, device=dev)
 
     def step():
-        for x, w8, y, ws in calls:
-            tw2.linear_i8(x, w8, y, ws, flags=flags)
+        call(ws, flags=flags)
 
     step()
     torch.cuda.synchronize()
@@ -589,13 +590,13 @@ def run_i8_decode(dev, stream, flags, world):
         raise RuntimeError(f"device flags {int(flags.item())} in the I8_S run")
     hbm, _, _ = _peaks()
     gbs = weight_bytes / (t * 1e-3) / 1e9
-    return {"workload": "I8_S decode, M=1, %d decoder layers x seven linears with int8 weights (%.1f MB > L2)"
-                        % (I8_LAYERS, weight_bytes / 1e6),
+    return {"workload": "I8_S decode, M=1, %d decoder layers x seven linears with int8 weights (%.1f MB > L2), "
+                        "one grouped call" % (I8_LAYERS, weight_bytes / 1e6),
             "tokens_per_s": round(whole_job_rate(world, 1, t), 1), "ms_per_step": round(t, 5),
-            "launches_per_step": 2 * len(calls),
+            "launches_per_step": len(xs) + 1,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "bytes_per_weight": 1.0},
-            "kernels": "quant_kernel + i8_gemv_kernel<1> per linear"}
+            "kernels": "quant_kernel per distinct input + one i8_gemv_kernel<1> over all rows"}
 
 
 def build_stack_views(m, dev, tws, layers=28):

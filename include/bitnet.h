@@ -341,6 +341,25 @@ BITNET_API bitnet_status bitnet_linear_i8(const float *x, int64_t m, const bitne
                                           int32_t *d_flags, void *stream);
 
 /*
+ * `count` I8_S layers sharing the token count m in one GEMV launch per slice
+ * of at most 8 tokens (the decoder-layer pattern: several linears, some on
+ * the same input).  Distinct inputs (same x pointer and k) are quantised
+ * once each into the workspace, then one launch streams the rows of all the
+ * layers.  Arguments as bitnet_linear_i8, per layer: x[i], w[i], y[i],
+ * acc_out (NULL or an array of `count` entries that may be NULL), epi (NULL
+ * or an array of `count` descriptors).  workspace >=
+ * bitnet_linear_i8_grouped_workspace_bytes(x, m, w, count), 256-byte
+ * aligned.  1 <= count <= BITNET_I8_GROUP_MAX.
+ */
+#define BITNET_I8_GROUP_MAX 64
+BITNET_API size_t bitnet_linear_i8_grouped_workspace_bytes(const float *const *x, int64_t m, const bitnet_i8w *w,
+                                                           int64_t count);
+BITNET_API bitnet_status bitnet_linear_i8_grouped(const float *const *x, int64_t m, const bitnet_i8w *w,
+                                                  const bitnet_epilogue *epi, int64_t count, float *const *y,
+                                                  int32_t *const *acc_out, void *workspace, size_t workspace_bytes,
+                                                  int32_t *d_flags, void *stream);
+
+/*
  * bitnet_linear_stack with no device allocation, for callers that cannot call
  * cudaMalloc: code running where the allocator is owned by someone else (a
  * host framework with its own pooling allocator, a real-time loop that must not

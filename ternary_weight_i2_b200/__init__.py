@@ -5,7 +5,7 @@ The compute lives in ``libbitnet.so`` (CUDA kernels behind the C ABI of
 used by callers for device memory and streams.
 """
 from ._abi import (  # noqa: F401
-    BitnetError, Epilogue, I8W, StackCall, TW, make_epilogue, make_i8w, linear_i8, i8_row_bytes,
+    BitnetError, Epilogue, I8GroupCall, I8W, StackCall, TW, make_epilogue, make_i8w, linear_i8, i8_row_bytes,
     linear_i8_workspace_bytes, header_functions, kpad, linear, linear_q, linear_stack,
     linear_stack_noalloc, linear_q_grouped, GroupedCall,
     linear_workspace_bytes, load, make_tw, pack_ternary, packed_bytes, quant_act,

@@ -73,6 +73,9 @@ _SIGNATURES = {
     "bitnet_i8_row_bytes": ([_I64], C.c_size_t),
     "bitnet_linear_i8_workspace_bytes": ([_I64, _I64], C.c_size_t),
     "bitnet_linear_i8": ([_P, _I64, C.POINTER(I8W), C.POINTER(Epilogue), _P, _P, _P, C.c_size_t, _P, _P], C.c_int),
+    "bitnet_linear_i8_grouped_workspace_bytes": ([_P, _I64, C.POINTER(I8W), _I64], C.c_size_t),
+    "bitnet_linear_i8_grouped": ([_P, _I64, C.POINTER(I8W), C.POINTER(Epilogue), _I64, _P, _P, _P, C.c_size_t,
+                                  _P, _P], C.c_int),
     "bitnet_debug_set_wait_limit": ([C.c_uint64], C.c_int),
     "bitnet_debug_force_stall": ([C.c_int], C.c_int),
     "bitnet_debug_set_trace": ([_P], C.c_int),
@@ -241,6 +244,33 @@ def linear_i8(x, w8: I8W, y, workspace, acc=None, flags=None, stream=None, epi: 
     _check(load().bitnet_linear_i8(_ptr(x), m, C.byref(w8), None if epi is None else C.byref(epi), _ptr(y),
                                    _ptr(acc), _ptr(workspace), ws_bytes, _ptr(flags), _stream(stream)),
            "bitnet_linear_i8")
+
+
+class I8GroupCall:
+    """Marshalled arguments of one bitnet_linear_i8_grouped call (reusable);
+    ``workspace_bytes`` is what the call needs."""
+
+    def __init__(self, xs, w8s, ys, accs=None, epis=None):
+        count = len(w8s)
+        self.count = count
+        self.m = xs[0].shape[0]
+        self.x_arr = (C.c_void_p * count)(*[x.data_ptr() for x in xs])
+        self.y_arr = (C.c_void_p * count)(*[y.data_ptr() for y in ys])
+        self.w_arr = (I8W * count)(*w8s)
+        self.acc_arr = None
+        if accs is not None:
+            self.acc_arr = (C.c_void_p * count)(*[(a.data_ptr() if a is not None else None) for a in accs])
+        self.epi_arr = None if epis is None else (Epilogue * count)(*[e if e is not None else Epilogue()
+                                                                      for e in epis])
+        self.workspace_bytes = int(load().bitnet_linear_i8_grouped_workspace_bytes(self.x_arr, self.m, self.w_arr,
+                                                                                   count))
+        self._keep = (xs, ys, accs)
+
+    def __call__(self, workspace, flags=None, stream=None) -> None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+        _check(load().bitnet_linear_i8_grouped(self.x_arr, self.m, self.w_arr, self.epi_arr, self.count, self.y_arr,
+                                               self.acc_arr, _ptr(workspace), ws_bytes, _ptr(flags),
+                                               _stream(stream)), "bitnet_linear_i8_grouped")
 
 
 def linear_q(xq, act_scale, tw: TW, y, acc=None, flags=None, stream=None, epi: Epilogue | None = None) -> None:

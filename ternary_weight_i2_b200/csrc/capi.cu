@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "gemv_i8.cuh"
 #include "gemv.cuh"
 
 namespace bitnet {
@@ -26,6 +27,7 @@ bool gemm_available();
 cudaError_t launch_gemv_i8(const int8_t *w, int64_t n, int64_t k, float s_w, const int8_t *q, const float *s_act,
                            int64_t m, const bitnet_epilogue *e, float *y, int32_t *acc, int sm_count,
                            cudaStream_t st);
+
 cudaError_t launch_gemm(const int8_t *xq, const float *act_scale, int64_t m, const bitnet_tw *w,
                         const bitnet_epilogue *epi, float *y, int32_t *acc, int32_t *flags, uint64_t wait_limit,
                         int force_stall, int sm_count, uint64_t *trace, cudaStream_t st);
@@ -815,6 +817,113 @@ size_t bitnet_linear_i8_workspace_bytes(int64_t m, int64_t k)
     if (m < 1 || m > (int64_t(1) << 31) - 1 || k < 1 || k > BITNET_MAX_K) return 0;
     const size_t a = size_t(m) * size_t(128 * blocks_of(k));
     return (a + 255) / 256 * 256 + size_t(m) * sizeof(float);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace layout of a grouped I8_S call: for each distinct input (same x
+// pointer and k, in order of first use) its int8 rows [m, kpad] and then its
+// scales [m], each area rounded up to 256 bytes.  input_of[i] = the distinct
+// input of layer i; offsets of its two areas in q_off / s_off.
+struct I8Plan {
+    std::vector<int> input_of;
+    std::vector<size_t> q_off, s_off;
+    std::vector<int64_t> first;   // a layer that uses the input
+    size_t bytes = 0;
+};
+
+void plan_i8(const float *const *x, int64_t m, const bitnet_i8w *w, int64_t count, I8Plan &P)
+{
+    P.input_of.assign(size_t(count), -1);
+    P.q_off.clear();
+    P.s_off.clear();
+    P.first.clear();
+    size_t off = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        int found = -1;
+        for (size_t j = 0; j < P.first.size(); ++j)
+            if (x[P.first[j]] == x[i] && w[P.first[j]].k == w[i].k) found = int(j);
+        if (found < 0) {
+            found = int(P.first.size());
+            P.first.push_back(i);
+            const size_t qa = size_t(m) * size_t(128 * blocks_of(w[i].k));
+            P.q_off.push_back(off);
+            off += (qa + 255) / 256 * 256;
+            P.s_off.push_back(off);
+            off += (size_t(m) * sizeof(float) + 255) / 256 * 256;
+        }
+        P.input_of[size_t(i)] = found;
+    }
+    P.bytes = off;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_linear_i8_grouped_workspace_bytes(const float *const *x, int64_t m, const bitnet_i8w *w, int64_t count)
+{
+    if (!x || !w || count < 1 || count > BITNET_I8_GROUP_MAX || m < 1 || m > (int64_t(1) << 31) - 1) return 0;
+    for (int64_t i = 0; i < count; ++i)
+        if (w[i].k < 1 || w[i].k > BITNET_MAX_K) return 0;
+    I8Plan P;
+    plan_i8(x, m, w, count, P);
+    return P.bytes;
+}
+
+bitnet_status bitnet_linear_i8_grouped(const float *const *x, int64_t m, const bitnet_i8w *w,
+                                       const bitnet_epilogue *epi, int64_t count, float *const *y,
+                                       int32_t *const *acc_out, void *workspace, size_t workspace_bytes,
+                                       int32_t *d_flags, void *stream)
+{
+    if (!x || !w || !y) return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: NULL array");
+    if (count < 1 || count > BITNET_I8_GROUP_MAX)
+        return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: count=%lld out of range [1, %d]", (long long)count,
+                    BITNET_I8_GROUP_MAX);
+    if (m < 1 || m > (int64_t(1) << 31) - 1) return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: bad m");
+    for (int64_t i = 0; i < count; ++i) {
+        if (!x[i] || !y[i] || !w[i].w)
+            return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: layer %lld has a NULL pointer", (long long)i);
+        if (w[i].n < 1 || w[i].n > (int64_t(1) << 30) || w[i].k < 1 || w[i].k > BITNET_MAX_K)
+            return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: layer %lld bad sizes", (long long)i);
+        if (!aligned(w[i].w, 16) || !aligned(x[i], 16))
+            return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: layer %lld weights or x not 16-byte aligned",
+                        (long long)i);
+        if (epi) {
+            bitnet_status s = check_epi(epi + i, i);
+            if (s != BITNET_OK) return s;
+        }
+    }
+    static thread_local I8Plan P;
+    plan_i8(x, m, w, count, P);
+    if (!workspace || workspace_bytes < P.bytes)
+        return fail(BITNET_ERR_WORKSPACE, "linear_i8_grouped: workspace of %zu bytes needed, %zu given", P.bytes,
+                    workspace_bytes);
+    if (!aligned(workspace, 256))
+        return fail(BITNET_ERR_INVALID_ARG, "linear_i8_grouped: workspace not 256-byte aligned");
+    DevInfo dev;
+    bitnet_status s = check_device(&dev);
+    if (s != BITNET_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    for (size_t j = 0; j < P.first.size(); ++j) {
+        const int64_t i = P.first[j];
+        cudaError_t e = launch_quant(x[i], m, w[i].k, reinterpret_cast<int8_t *>(ws + P.q_off[j]),
+                                     reinterpret_cast<float *>(ws + P.s_off[j]), d_flags, st);
+        if (e != cudaSuccess) return cuda_fail(e, "quant launch");
+    }
+    static thread_local std::vector<I8Job> jobs;
+    jobs.resize(size_t(count));
+    for (int64_t i = 0; i < count; ++i) {
+        const int j = P.input_of[size_t(i)];
+        jobs[size_t(i)] = I8Job{w[i].w, w[i].n, w[i].k, w[i].scale, reinterpret_cast<const int8_t *>(ws + P.q_off[j]),
+                                reinterpret_cast<const float *>(ws + P.s_off[j]), y[i],
+                                acc_out ? acc_out[i] : nullptr, epi ? epi + i : nullptr};
+    }
+    cudaError_t e = launch_gemv_i8_group(jobs.data(), int(count), m, dev.sm_count, st);
+    return e == cudaSuccess ? BITNET_OK : cuda_fail(e, "i8 gemv launch");
 }
 
 bitnet_status bitnet_linear_i8(const float *x, int64_t m, const bitnet_i8w *w, const bitnet_epilogue *epi, float *y,

@@ -17,27 +17,52 @@
 // a [m, kpad] int8 buffer) are read through L1.  No shared-memory pipeline
 // and no waits.
 #include "common.cuh"
+#include "gemv_i8.cuh"
 
 namespace bitnet {
 
 constexpr int kI8Warps = 8;          // warps (rows in flight) per CTA
 constexpr int kI8CtasPerSm = 8;
 
-struct I8Epilogue {
+constexpr int kI8MaxGroup = 64;     // linears per grouped launch
+
+// One linear of a launch: its weights, this token slice's activations and
+// outputs, and its epilogue operands.
+struct I8Linear {
+    const int8_t *w;
+    const int8_t *q;          // int8 activations [MT, kpad] of this slice
+    const float *s_act;       // [MT]
+    float *y;                 // [MT, n] of this slice
+    int32_t *acc;             // [MT, n] or null
     const float *bias, *gamma, *res;
-    int relu;
+    int64_t n, rowb, kpad;
+    int64_t row0;             // first row of this linear in the launch's row numbering
+    float s_w;
+    int32_t relu;
 };
 
+struct I8Params {
+    int32_t count;
+    int64_t total_rows;
+    I8Linear lin[kI8MaxGroup];
+};
+static_assert(sizeof(I8Params) <= 32760, "I8_S parameter block too large");
+
+// The rows of all the launch's linears form one numbering; warps take rows
+// of it round-robin.
 template <int MT>
-__global__ void __launch_bounds__(kI8Warps * 32) i8_gemv_kernel(const int8_t *__restrict__ w, int64_t n,
-                                                             int64_t rowb, const int8_t *__restrict__ q,
-                                                             int64_t kpad, const float *__restrict__ s_act,
-                                                             float s_w, I8Epilogue epi, float *y, int32_t *acc_out)
+__global__ void __launch_bounds__(kI8Warps * 32) i8_gemv_kernel(const __grid_constant__ I8Params p)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t chunks = rowb / 16;            // 16-byte chunks per row
-    for (int64_t row = int64_t(blockIdx.x) * kI8Warps + warp; row < n; row += int64_t(gridDim.x) * kI8Warps) {
-        const int4 *wr = reinterpret_cast<const int4 *>(w + row * rowb);
+    for (int64_t grow = int64_t(blockIdx.x) * kI8Warps + warp; grow < p.total_rows;
+         grow += int64_t(gridDim.x) * kI8Warps) {
+        int li = 0;
+        while (li + 1 < p.count && p.lin[li + 1].row0 <= grow) ++li;
+        const I8Linear &L = p.lin[li];
+        const int64_t row = grow - L.row0, n = L.n, rowb = L.rowb, kpad = L.kpad;
+        const int8_t *__restrict__ q = L.q;
+        const int64_t chunks = rowb / 16;        // 16-byte chunks per row
+        const int4 *wr = reinterpret_cast<const int4 *>(L.w + row * rowb);
         int32_t acc[MT];
 #pragma unroll
         for (int t = 0; t < MT; ++t) acc[t] = 0;
@@ -81,59 +106,76 @@ __global__ void __launch_bounds__(kI8Warps * 32) i8_gemv_kernel(const int8_t *__
         for (int t = 0; t < MT; ++t) {
             if (lane == t) {
                 const size_t o = size_t(t) * size_t(n) + size_t(row);
-                float v = __fmul_rn(__fmul_rn(float(acc[t]), s_act[t]), s_w);
-                if (epi.bias) v = __fadd_rn(v, epi.bias[row]);
-                if (epi.relu) v = v > 0.f ? v : 0.f;
-                if (epi.gamma) v = __fmul_rn(epi.gamma[row], v);
-                if (epi.res) v = __fadd_rn(epi.res[o], v);
-                y[o] = v;
-                if (acc_out) acc_out[o] = acc[t];
+                float v = __fmul_rn(__fmul_rn(float(acc[t]), L.s_act[t]), L.s_w);
+                if (L.bias) v = __fadd_rn(v, L.bias[row]);
+                if (L.relu) v = v > 0.f ? v : 0.f;
+                if (L.gamma) v = __fmul_rn(L.gamma[row], v);
+                if (L.res) v = __fadd_rn(L.res[o], v);
+                L.y[o] = v;
+                if (L.acc) L.acc[o] = acc[t];
             }
         }
     }
 }
 
-template <int MT>
-static cudaError_t launch_mt(const int8_t *w, int64_t n, int64_t rowb, const int8_t *q, int64_t kpad,
-                             const float *s_act, float s_w, I8Epilogue epi, float *y, int32_t *acc, int grid,
-                             cudaStream_t st)
-{
-    i8_gemv_kernel<MT><<<grid, kI8Warps * 32, 0, st>>>(w, n, rowb, q, kpad, s_act, s_w, epi, y, acc);
-    return cudaGetLastError();
-}
+static_assert(kI8MaxGroup == BITNET_I8_GROUP_MAX, "group limit");
 
-// Quantised activations q [m, kpad] and scales [m] are already in device
-// memory; runs the tokens in slices of at most 8.
-cudaError_t launch_gemv_i8(const int8_t *w, int64_t n, int64_t k, float s_w, const int8_t *q, const float *s_act,
-                           int64_t m, const bitnet_epilogue *e, float *y, int32_t *acc, int sm_count,
-                           cudaStream_t st)
+cudaError_t launch_gemv_i8_group(const I8Job *jobs, int count, int64_t m, int sm_count, cudaStream_t st)
 {
-    const int64_t rowb = 32 * ((k + 31) / 32), kpad = 128 * ((k + 127) / 128);
-    const int64_t want = (n + kI8Warps - 1) / kI8Warps;
+    if (count < 1 || count > kI8MaxGroup) return cudaErrorInvalidValue;
+    static thread_local I8Params p;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) total += jobs[i].n;
+    const int64_t want = (total + kI8Warps - 1) / kI8Warps;
     const int64_t cap = int64_t(sm_count) * kI8CtasPerSm;
     const int grid = int(want < cap ? want : cap);
     for (int64_t m0 = 0; m0 < m; m0 += 8) {
         const int mt = int(m - m0 < 8 ? m - m0 : 8);
-        I8Epilogue epi{nullptr, nullptr, nullptr, 0};
-        if (e) epi = I8Epilogue{e->bias, e->gamma, e->residual ? e->residual + m0 * n : nullptr, e->relu ? 1 : 0};
-        const int8_t *qs = q + m0 * kpad;
-        const float *ss = s_act + m0;
-        float *ys = y + m0 * n;
-        int32_t *as = acc ? acc + m0 * n : nullptr;
-        cudaError_t r;
-        switch (mt) {
-        case 1: r = launch_mt<1>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 2: r = launch_mt<2>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 3: r = launch_mt<3>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 4: r = launch_mt<4>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 5: r = launch_mt<5>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 6: r = launch_mt<6>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        case 7: r = launch_mt<7>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
-        default: r = launch_mt<8>(w, n, rowb, qs, kpad, ss, s_w, epi, ys, as, grid, st); break;
+        p.count = count;
+        p.total_rows = total;
+        int64_t row0 = 0;
+        for (int i = 0; i < count; ++i) {
+            const I8Job &J = jobs[i];
+            I8Linear &L = p.lin[i];
+            L.w = J.w;
+            L.n = J.n;
+            L.rowb = 32 * ((J.k + 31) / 32);
+            L.kpad = 128 * ((J.k + 127) / 128);
+            L.q = J.q + m0 * L.kpad;
+            L.s_act = J.s_act + m0;
+            L.y = J.y + m0 * J.n;
+            L.acc = J.acc ? J.acc + m0 * J.n : nullptr;
+            L.bias = J.epi ? J.epi->bias : nullptr;
+            L.gamma = J.epi ? J.epi->gamma : nullptr;
+            L.res = (J.epi && J.epi->residual) ? J.epi->residual + m0 * J.n : nullptr;
+            L.relu = (J.epi && J.epi->relu) ? 1 : 0;
+            L.s_w = J.s_w;
+            L.row0 = row0;
+            row0 += J.n;
         }
+        const dim3 blk(kI8Warps * 32);
+        switch (mt) {
+        case 1: i8_gemv_kernel<1><<<grid, blk, 0, st>>>(p); break;
+        case 2: i8_gemv_kernel<2><<<grid, blk, 0, st>>>(p); break;
+        case 3: i8_gemv_kernel<3><<<grid, blk, 0, st>>>(p); break;
+        case 4: i8_gemv_kernel<4><<<grid, blk, 0, st>>>(p); break;
+        case 5: i8_gemv_kernel<5><<<grid, blk, 0, st>>>(p); break;
+        case 6: i8_gemv_kernel<6><<<grid, blk, 0, st>>>(p); break;
+        case 7: i8_gemv_kernel<7><<<grid, blk, 0, st>>>(p); break;
+        default: i8_gemv_kernel<8><<<grid, blk, 0, st>>>(p); break;
+        }
+        cudaError_t r = cudaGetLastError();
         if (r != cudaSuccess) return r;
     }
     return cudaSuccess;
+}
+
+cudaError_t launch_gemv_i8(const int8_t *w, int64_t n, int64_t k, float s_w, const int8_t *q, const float *s_act,
+                           int64_t m, const bitnet_epilogue *e, float *y, int32_t *acc, int sm_count,
+                           cudaStream_t st)
+{
+    const I8Job j{w, n, k, s_w, q, s_act, y, acc, e};
+    return launch_gemv_i8_group(&j, 1, m, sm_count, st);
 }
 
 }  // namespace bitnet

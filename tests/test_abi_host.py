@@ -162,3 +162,26 @@ def test_epilogue_forms_report_no_device(lib):
     st = lib.bitnet_quantize_pack(P(0x10000), 4, 4, P(0x20000), P(0x30000), P(0x40000),
                                   lib.bitnet_quantize_pack_workspace_bytes(), None, None)
     assert st in (_abi.ERR_CUDA, _abi.ERR_UNSUPPORTED_DEVICE)
+
+
+def test_i8_sizes_and_grouped_workspace_layout(lib):
+    assert tw2.i8_row_bytes(1) == 32 and tw2.i8_row_bytes(1536) == 1536 and tw2.i8_row_bytes(8961) == 8992
+    assert tw2.i8_row_bytes(0) == 0 and tw2.i8_row_bytes(65537) == 0
+    assert tw2.linear_i8_workspace_bytes(1, 1536) == 1536 + 4
+    # inputs are shared when both the pointer and k match: A(1536), A(1536),
+    # B(8960) and A(8960) are three distinct inputs
+    xs = (C.c_void_p * 4)(0x10000, 0x10000, 0x20000, 0x10000)
+    ws = (_abi.I8W * 4)(_abi.I8W(0x1000, 8, 1536, 1.0), _abi.I8W(0x1000, 8, 1536, 1.0),
+                        _abi.I8W(0x1000, 8, 8960, 1.0), _abi.I8W(0x1000, 8, 8960, 1.0))
+    per = {1536: 1536 + 256, 8960: 8960 + 256}   # int8 rows [1, kpad] then scales, each rounded to 256 bytes
+    assert lib.bitnet_linear_i8_grouped_workspace_bytes(xs, 1, ws, 4) == per[1536] + 2 * per[8960]
+    assert lib.bitnet_linear_i8_grouped_workspace_bytes(xs, 1, ws, 2) == per[1536]
+    assert lib.bitnet_linear_i8_grouped_workspace_bytes(xs, 1, ws, 65) == 0
+    # argument checks before any device call
+    ys = (C.c_void_p * 4)(0x30000, 0x40000, 0x50000, 0x60000)
+    big = lib.bitnet_linear_i8_grouped_workspace_bytes(xs, 1, ws, 4)
+    assert lib.bitnet_linear_i8_grouped(xs, 1, ws, None, 4, ys, None, C.c_void_p(0x100000), big - 1, None,
+                                        None) == _abi.ERR_WORKSPACE
+    bad = (_abi.I8W * 1)(_abi.I8W(0x1008, 8, 1536, 1.0))
+    assert lib.bitnet_linear_i8_grouped(xs, 1, bad, None, 1, ys, None, C.c_void_p(0x100000), big, None,
+                                        None) == _abi.ERR_INVALID_ARG

@@ -108,3 +108,45 @@ def test_linear_i8_fused_epilogue(m):
     o32, _ = oracle.epilogue(y32, bias=b, gamma=g, residual=r, relu=True)
     np.testing.assert_array_equal(ag, acc)
     np.testing.assert_array_equal(yg.view(np.uint32), o32.view(np.uint32))
+
+
+@pytest.mark.parametrize("m", [1, 13])
+def test_linear_i8_grouped_decoder_layer(m):
+    """One decoder layer's seven linears in one grouped call (the four
+    distinct inputs quantised once each, one GEMV launch per 8-token slice),
+    epilogues on some layers: every layer against the oracle."""
+    rng = np.random.default_rng(500 + m)
+    xs_host = synth.layer_inputs(0, m, 2)
+    xdev = [upload(a) for a in xs_host]
+    w8s, keep, ys, accs, epis, ref = [], [], [], [], [], []
+    for i, ((name, n, k), j) in enumerate(zip(synth.LAYER_SHAPES, synth.LAYER_INPUT_OF)):
+        rows = _weights(rng, n, k)
+        s_w = synth.weight_scale(rng)
+        wd = upload(rows)
+        keep.append(wd)
+        w8s.append(tw2.make_i8w(wd, n, k, s_w))
+        ys.append(Guarded((m, n), torch.float32))
+        accs.append(Guarded((m, n), torch.int32))
+        if i % 2 == 0:
+            b = rng.standard_normal(n).astype(np.float32)
+            r = rng.standard_normal((m, n)).astype(np.float32)
+            bd, rd = upload(b), upload(r)
+            keep.append((bd, rd))
+            epis.append(tw2.make_epilogue(bias=bd, residual=rd, relu=(i == 4)))
+            ref.append((xs_host[j], rows, k, s_w, b, r, i == 4))
+        else:
+            epis.append(None)
+            ref.append((xs_host[j], rows, k, s_w, None, None, False))
+    call = tw2.I8GroupCall([xdev[j] for j in synth.LAYER_INPUT_OF], w8s, [y.t for y in ys], [a.t for a in accs],
+                           epis=epis)
+    ws = torch.empty(call.workspace_bytes, dtype=torch.uint8, device=DEV)
+    fl = flags_tensor()
+    call(ws, flags=fl)
+    torch.cuda.synchronize()
+    assert int(fl.item()) == 0
+    for y, a, (x, rows, k, s_w, b, r, relu) in zip(ys, accs, ref):
+        assert y.guard_intact() and a.guard_intact()
+        acc, y64, y32, _ = oracle.linear_i8(x, rows, k, s_w)
+        o32, _ = oracle.epilogue(y32, bias=b, residual=r, relu=relu)
+        np.testing.assert_array_equal(a.t.cpu().numpy(), acc)
+        np.testing.assert_array_equal(y.t.cpu().numpy().view(np.uint32), o32.view(np.uint32))
