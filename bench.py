@@ -366,6 +366,10 @@ def run_gpu(args):
         prefill = run_prefill(dev, stream, flags, world)
     qpack = run_quantize_pack(dev, stream, flags, world)
     i8_line = run_i8_decode(dev, stream, flags, world)
+    try:
+        pack_line = run_pack(dev, stream, flags, world)
+    except Exception as e:   # a load-time side measurement must not cost the main line
+        pack_line = {"error": str(e)[:300]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -395,6 +399,7 @@ def run_gpu(args):
             "quantize_pack": qpack,
             "fused_epilogue_stack": epi_line,
             "i8s_decode": i8_line,
+            "pack": pack_line,
         }
         print(json.dumps(line))
     if world > 1:
@@ -459,6 +464,9 @@ def run_prefill(dev, stream, flags, world):
     tq, _ = time_device(gq.replay, 20, 3, stream)
     tg, per = time_device(gg.replay, 20, 3, stream)
     tq, tg = _max_over_ranks(tq) / 20, _max_over_ranks(tg) / 20
+    # the quantiser's algorithmic bytes: fp32 in, int8 rows (with pads) and
+    # one fp32 scale per token out, per distinct input
+    quant_bytes = sum(PREFILL_M * (4 * k + tw2.kpad(k) + 4) for k in xs)
     # the same launch with the fused epilogue on every layer (bias, layer
     # scale, residual add; ReLU on gate and up)
     epi_keep, epis = [], []
@@ -495,7 +503,12 @@ def run_prefill(dev, stream, flags, world):
             "roofline": {"bound": "tensor", "achieved": round(tops / world, 1), "peak": round(peak, 1),
                          "unit": "TOPS", "frac": round(tops / world / peak, 4),
                          "peak_kind": "measured bf16 cuBLAS burst (MEASURED_PEAKS.json) x 2 (int8:bf16 dense ratio)"},
-            "quant_ms_per_step": round(tq, 5), "per_shape": per_shape,
+            "quant_ms_per_step": round(tq, 5),
+            "quant_roofline": {"bound": "hbm", "achieved": round(quant_bytes / (tq * 1e-3) / 1e9, 1),
+                               "peak": round(_peaks()[0], 1), "unit": "GB/s",
+                               "frac": round(quant_bytes / (tq * 1e-3) / 1e9 / _peaks()[0], 4),
+                               "bytes": quant_bytes, "kernel": "quant_kernel (a2 standalone)"},
+            "per_shape": per_shape,
             "with_fused_epilogue": {"ms_per_step": round(te, 5),
                                     "tops": round(whole_job_rate(world, PREFILL_OPS, te) / 1e12, 1),
                                     "epilogue": "bias + layer scale + residual add on all seven (ReLU on gate/up)"},
@@ -549,6 +562,49 @@ def run_quantize_pack(dev, stream, flags, world):
 
 
 I8_LAYERS = 4
+PACK_LAYERS = 4
+
+
+def run_pack(dev, stream, flags, world):
+    """Load-time pack (int8 ternary -> 2-bit codes) of four decoder layers'
+    28 tensors per step (187 MB of int8, larger than L2), graph-replayed.
+    Algorithmic bytes: 1 B read + 1/4 B written per weight."""
+    import torch
+    import ternary_weight_i2_b200 as tw2
+    from ternary_weight_i2_b200 import synth
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.seed_for(7, 0))
+    work, weights = [], 0
+    for L in range(PACK_LAYERS):
+        for name, n, k in synth.LAYER_SHAPES:
+            w = torch.randint(-1, 2, (n, k), generator=g, device=dev, dtype=torch.int8)
+            pk = torch.empty((n, tw2.packed_bytes(n, k) // n), dtype=torch.uint8, device=dev)
+            work.append((w, pk))
+            weights += n * k
+
+    def step():
+        for w, pk in work:
+            tw2.pack_ternary(w, pk, flags=flags)
+
+    step()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        step()
+    steps = 10
+    t, _ = time_device(gr.replay, steps, 3, stream)
+    t = _max_over_ranks(t) / steps
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"device flags {int(flags.item())} in the pack run")
+    hbm, _, _ = _peaks()
+    gbs = 1.25 * weights / (t * 1e-3) / 1e9
+    return {"workload": "pack of %d decoder layers' %d ternary int8 tensors (%.1f MB > L2)"
+                        % (PACK_LAYERS, len(work), weights / 1e6),
+            "ms_per_step": round(t, 5), "launches_per_step": len(work),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "bytes_per_weight": 1.25},
+            "kernels": "pack_kernel"}
 
 
 def run_i8_decode(dev, stream, flags, world):

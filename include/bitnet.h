@@ -249,7 +249,7 @@ BITNET_API bitnet_status bitnet_linear_q(const int8_t *xq, const float *act_scal
  * `count` independent layers on pre-quantised activations in one launch
  * (prefill: the token count m is shared, each layer has its own input, weight
  * and output; TR §3.2, Figure 6a).  m > 8 runs one persistent tensor-core GEMM
- * over all layers' 128 x 256 output tiles, dealt to the SMs heaviest first, so
+ * over all layers' 128-feature x 192-token output tiles, dealt to the SMs heaviest first, so
  * that layers of different K and N balance inside one launch; m <= 8 runs the
  * streaming GEMV.
  *   xq[i]        device int8 [m, bitnet_kpad(w[i].k)], 16-byte aligned, pads 0

@@ -1,6 +1,6 @@
 """Parity of the prefill path (M > 8: per-token quantiser + tcgen05 int8 GEMM)
 with the CPU oracle, through the C ABI.  Full comparisons on shapes the oracle
-finishes in seconds (several 128 x 256 tiles and ragged tails); at the prefill
+finishes in seconds (several 128 x 192 tiles and ragged tails); at the prefill
 size (M = 2048 over the seven decoder-layer shapes, the launch bench.py times)
 every output is checked against its exact int32 sum by the dequantisation
 identity and sampled output columns against the oracle."""
