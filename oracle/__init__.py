@@ -199,6 +199,37 @@ def linear_i8(x, w_rows, k, s_w):
     return acc, y64, y32, st
 
 
+# Reading R8: the decoder layer's linears as a dependence chain.  The path
+# holds no attention, normalisation or activation op, so each is replaced by
+# the plainest stand-in of matching width: the attention output by q's
+# output, the gated activation by up's output.  Input of each linear, by
+# position in (q, k, v, o, gate, up, down): the layer input for q, k, v; q's
+# output for o; o's output for gate and up; up's output for down.  down's
+# output is the next layer's input.
+CHAIN_INPUT_OF = (-1, -1, -1, 0, 3, 3, 5)   # -1: the layer input
+
+
+def linear_chain(x0, layers):
+    """Decode chain (reading R8): ``layers`` is a list of decoder layers, each
+    a list of seven (packed, n, k, s_w) in (q, k, v, o, gate, up, down) order.
+    Every linear quantises its fp32 input (R1) and feeds its fp32 output (the
+    R4 fp32 form) forward.  Returns (outputs per layer as lists of y32 [m, n],
+    status)."""
+    x = _np.ascontiguousarray(x0, _np.float32)
+    outs, st = [], 0
+    for layer in layers:
+        ys = []
+        for i, (packed, n, k, s_w) in enumerate(layer):
+            src = x if CHAIN_INPUT_OF[i] < 0 else ys[CHAIN_INPUT_OF[i]]
+            assert src.shape[1] == k, "chain width mismatch"
+            _, _, y32, s1 = linear(src, packed, n, k, s_w)
+            ys.append(y32)
+            st |= s1
+        outs.append(ys)
+        x = ys[6]
+    return outs, st
+
+
 def linear_rows(x, packed, n, k, s_w, rows):
     """Only the output columns ``rows`` -> (acc int32 [m,cnt], y64 [m,cnt], status)."""
     x = _c(x, _np.float32)

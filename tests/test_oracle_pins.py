@@ -551,3 +551,61 @@ def test_linear_i8_fp32_form_rounds_large_sums_to_even():
     assert acc[0, 0] == 16790289
     assert y64[0, 0] == 16790289.0
     assert y32[0, 0] == np.float32(16790288.0)
+
+
+# ---------------------------------------------------- decode chain (R8)
+
+def _identity_like(n, k, sign=1):
+    w = np.zeros((n, k), np.int8)
+    d = min(n, k)
+    w[np.arange(d), np.arange(d)] = sign
+    return w
+
+
+def _chain_layers(shapes_weights, s_w=1.0):
+    return [[(oracle.pack(w)[0], w.shape[0], w.shape[1], s_w) for w in layer] for layer in shapes_weights]
+
+
+def test_chain_carries_codes_only_along_the_true_dependences():
+    """Identity weights on the chain's true path (q -> o -> up -> down) and
+    zero weights elsewhere (k, v, gate): the codes of the first input come
+    back out of every layer's down unchanged, times its scale.  A chain wired
+    through k, v or gate would give zeros."""
+    rng = np.random.default_rng(81)
+    x0 = synth.normal_outliers(rng, 2, 1536)
+    layer = [_identity_like(1536, 1536), np.zeros((256, 1536), np.int8), np.zeros((256, 1536), np.int8),
+             _identity_like(1536, 1536), np.zeros((8960, 1536), np.int8), _identity_like(8960, 1536),
+             _identity_like(1536, 8960)]
+    outs, st = oracle.linear_chain(x0, _chain_layers([layer, layer, layer]))
+    assert st == oracle.OK
+    q0, s0, _ = oracle.quant_act(x0)
+    for ys in outs:
+        qd, sd, _ = oracle.quant_act(ys[6])
+        np.testing.assert_array_equal(qd[:, :1536], q0[:, :1536])
+        assert not ys[1].any() and not ys[2].any() and not ys[4].any()
+        assert (np.abs(ys[6]) > 0).any()
+        # down's output is the first codes dequantised: within a few fp32
+        # roundings of q0 * s0 (s_w = 1 everywhere)
+        np.testing.assert_allclose(ys[6], q0[:, :1536] * s0[:, None], rtol=1e-5, atol=0)
+
+
+def test_chain_negating_the_first_linear_negates_everything_downstream():
+    """The quantiser is odd (rint is symmetric) and every later linear is
+    linear with the same scales, so flipping q's weights flips every later
+    output bit for bit in magnitude and exactly in sign."""
+    rng = np.random.default_rng(82)
+    x0 = synth.normal_outliers(rng, 1, 1536)
+    rest = [synth.ternary(rng, n, k) for _, n, k in synth.LAYER_SHAPES[1:]]
+    wq = synth.ternary(rng, 1536, 1536)
+    scales = [synth.weight_scale(rng) for _ in range(7)]
+
+    def run(wq_):
+        ws = [wq_] + rest
+        layer = [(oracle.pack(w)[0], w.shape[0], w.shape[1], s) for w, s in zip(ws, scales)]
+        return oracle.linear_chain(x0, [layer])[0][0]
+
+    a, b = run(wq), run(-wq)
+    for i in (0, 3, 4, 5, 6):      # q and everything that depends on it
+        np.testing.assert_array_equal(b[i], -a[i])
+    for i in (1, 2):               # k and v read the layer input only
+        np.testing.assert_array_equal(b[i], a[i])
