@@ -380,7 +380,7 @@ def run_gpu(args):
             "metric": METRIC, "value": round(tok_s, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
-            "data": "synthetic (seeded ternary weights and fp32 activations, BASELINE shapes)",
+            "data": "synthetic (seeded ternary weights and fp32 activations of the 1.5B-class decoder-layer shapes)",
             "config": {"workload": "%d-layer ternary linear stack, %d layers, M=%d decode"
                                    % (args.layers, 7 * args.layers, m),
                        "tokens_per_step_per_gpu": m, "layers": 7 * args.layers,
