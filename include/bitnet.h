@@ -10,13 +10,19 @@
  * run time, multiplied against the ternary weights with exact int32
  * accumulation, and the sums are dequantised in fp32.
  *
+ * Around it: the absmean quantiser that turns full-precision weights into
+ * the ternary codes and scale (bitnet_quantize_pack), an optional fused
+ * epilogue after the dequantisation (bias, ReLU, layer-scaled residual add:
+ * the operator fusion of §2.4.1; the *_ex entry points), and the I8_S layer
+ * with plain int8 weights (§2.2.1, §2.4.2; bitnet_linear_i8*).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Pointers named d_* or documented "device" point to CUDA device memory of
  *   the current device; the caller owns every buffer.  Functions that take a
  *   workspace never allocate; no function allocates device memory per call.
- *   The GEMV path (bitnet_linear with m <= 8, bitnet_linear_q with m <= 8,
- *   bitnet_linear_stack) streams each weight tensor through a TMA tensor map
+ *   The GEMV path (bitnet_linear[_ex] and bitnet_linear_q[_ex] with m <= 8,
+ *   bitnet_linear_stack[_ex]) streams each weight tensor through a TMA tensor map
  *   that the library encodes the first time it meets that tensor (same
  *   packed pointer, n and k) and keeps in a per-device cache (128 bytes of
  *   device memory per tensor, allocated 128 KB at a time, until
@@ -77,7 +83,8 @@ typedef enum {
     BITNET_ERR_NOT_TERNARY = 2,        /* a weight outside {-1,0,+1} (device flag)      */
     BITNET_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 (B200)           */
     BITNET_ERR_CUDA = 4,               /* a CUDA runtime call failed                    */
-    BITNET_ERR_NONFINITE = 5,          /* an activation row held NaN/Inf (device flag)  */
+    BITNET_ERR_NONFINITE = 5,          /* NaN/Inf in an activation row or in a weight
+                                          tensor being quantised (device flag)          */
     BITNET_ERR_TIMEOUT = 6,            /* a bounded device-side wait ran out (flag)     */
     BITNET_ERR_WORKSPACE = 7           /* the workspace given is too small              */
 } bitnet_status;
